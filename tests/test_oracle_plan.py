@@ -1,0 +1,170 @@
+"""Pins for the oracle's planner: hand-worked golden plans, an independent
+brute-force planner over exhaustive and random tiny routings, closed forms,
+and the plan invariants on the five workloads' routings."""
+import itertools
+
+import numpy as np
+import pytest
+
+from golden_io import load_plans
+from plan_bruteforce import brute_plan, check_plan_invariants
+from dispatch_moonep_plan_b200 import workloads as wl
+
+
+def _cmp_with_brute(oracle, idx, R, S, E, K, B, rule):
+    got = oracle.plan(R, S, E, K, B, idx, rule=rule)
+    ref = brute_plan(np.asarray(idx).reshape(R * S, K), R, S, E, K, B, rule)
+    assert got["status"] == ref["status"], (idx, got["status"], ref["status"])
+    if ref["status"] == 4:
+        return got
+    assert list(got["expert_count"]) == ref["expert_count"]
+    assert list(got["rank_load"]) == ref["rank_load"]
+    assert got["max_count"] == ref["max_count"]
+    assert got["maxvio"] == ref["maxvio"]
+    if ref["status"] == 3:
+        assert got["fail_rank"] == ref["fail_rank"]
+        assert got["fail_slots"] == ref["fail_slots"]
+        return got
+    assert got["slot_expert"].tolist() == ref["slot_expert"]
+    assert got["cu_seqlens"].tolist() == ref["cu_seqlens"]
+    assert got["dst_row"].tolist() == ref["dst_row"]
+    assert got["src_of_row"].tolist() == ref["src_of_row"]
+    return got
+
+
+@pytest.mark.parametrize("case", load_plans(), ids=lambda c: c["name"])
+def test_golden_plans(oracle_mod, case):
+    R, S, E, K, B, rule = (case[k] for k in ("R", "S", "E", "K", "B", "rule"))
+    idx = np.array(case["idx"], np.int32)
+    got = oracle_mod.plan(R, S, E, K, B, idx, rule=rule)
+    assert got["status"] == case["status"]
+    if case["status"] == 4:
+        return
+    assert got["expert_count"].tolist() == case["expert_count"]
+    assert got["rank_load"].tolist() == case["rank_load"]
+    assert got["max_count"] == case["max_count"]
+    assert abs(got["maxvio"] - float(case["maxvio"])) < 1e-12
+    if case["status"] == 3:
+        assert got["fail_rank"] == case["fail_rank"]
+        assert got["fail_slots"] == case["fail_slots"]
+        return
+    assert got["slot_expert"].tolist() == case["slot_expert"]
+    assert got["cu_seqlens"].tolist() == case["cu_seqlens"]
+    assert got["dst_row"].tolist() == case["dst_row"]
+    assert got["src_of_row"].tolist() == case["src_of_row"]
+    # the brute-force planner agrees with the paper-worked case too
+    ref = brute_plan(idx, R, S, E, K, B, rule)
+    assert ref["dst_row"] == case["dst_row"]
+
+
+@pytest.mark.parametrize("rule", [0, 1])
+def test_exhaustive_distinct_R2_S2_E4_K2(oracle_mod, rule):
+    """Every routing of 4 tokens over 4 experts with 2 distinct picks, with
+    B = 1 (every plan fits: one over-full rank of two experts overflows at
+    most one expert), and every 4th routing again with B = 0 (any overflow
+    fails)."""
+    R, S, E, K = 2, 2, 4, 2
+    pairs = [p for p in itertools.permutations(range(E), K)]
+    n_ok = n_fail = 0
+    for i, combo in enumerate(itertools.product(pairs, repeat=R * S)):
+        idx = np.array(combo, np.int32)
+        B = 0 if i % 4 == 3 else 1
+        got = _cmp_with_brute(oracle_mod, idx, R, S, E, K, B, rule)
+        if got["status"] == 0:
+            n_ok += 1
+            check_plan_invariants(got, idx, R, S, E, K, B, rule)
+        else:
+            n_fail += 1
+    assert n_ok > 0 and n_fail > 0
+
+
+def test_sampled_duplicates_R2_S3_E4_K2(oracle_mod):
+    """Routings with repeated picks inside a token (allowed: every (t, k) is
+    its own row), R=2, S=3, E=4, K=2, B in {1, 2}."""
+    rng = np.random.default_rng(1)
+    R, S, E, K = 2, 3, 4, 2
+    for it in range(3000):
+        B = 1 + it % 2
+        idx = rng.integers(0, E, (R * S, K)).astype(np.int32)
+        got = _cmp_with_brute(oracle_mod, idx, R, S, E, K, B, it % 3 == 0)
+        if got["status"] == 0:
+            check_plan_invariants(got, idx, R, S, E, K, B)
+
+
+@pytest.mark.parametrize("rule", [0, 1])
+def test_random_small_configs(oracle_mod, rule):
+    rng = np.random.default_rng(100 + rule)
+    seen = set()
+    for it in range(400):
+        cfg = wl.random_small_cfg(rng)
+        R, S, E, K, B = (cfg[k] for k in ("R", "S", "E", "K", "B"))
+        idx, _ = wl.routing(cfg, seed=it)
+        got = _cmp_with_brute(oracle_mod, idx, R, S, E, K, B, rule)
+        seen.add(got["status"])
+        if got["status"] == 0:
+            check_plan_invariants(got, idx, R, S, E, K, B, rule)
+    assert seen >= {0, 3}
+
+
+def test_bad_index(oracle_mod):
+    idx = np.array([[0, 1], [5, 0]], np.int32)
+    assert oracle_mod.plan(1, 2, 4, 2, 1, idx)["status"] == 4
+    idx = np.array([[0, 1], [-1, 0]], np.int32)
+    assert oracle_mod.plan(1, 2, 4, 2, 1, idx)["status"] == 4
+
+
+def test_invalid_args(oracle_mod):
+    idx = np.zeros((6, 1), np.int32)
+    assert oracle_mod.plan(2, 3, 3, 1, 1, idx)["status"] == 1  # E % R != 0
+
+
+def test_round_robin_closed_form(oracle_mod):
+    """idx[t,k] = (t*K+k) mod E gives every expert P/E rows, so every rank
+    holds exactly C home rows: no overflow, no slot, and every home group has
+    C/Er rows."""
+    for (R, S, E, K) in [(2, 4, 4, 2), (4, 6, 8, 4), (8, 32, 64, 6), (3, 5, 6, 6)]:
+        B = 3
+        cfg = dict(R=R, S=S, E=E, K=K, routing="round_robin")
+        idx, _ = wl.routing(cfg)
+        got = oracle_mod.plan(R, S, E, K, B, idx)
+        assert got["status"] == 0
+        Er, C = E // R, S * K
+        assert got["maxvio"] == 0.0
+        assert np.all(got["slot_expert"] == -1)
+        for r in range(R):
+            expect = [0] * r * Er + [(i + 1) * C // Er for i in range(Er)] + [C] * (E - (r + 1) * Er + B)
+            assert got["cu_seqlens"][r].tolist() == expect
+        # token order inside each expert group, rank by rank
+        check_plan_invariants(got, idx, R, S, E, K, B)
+
+
+def test_maxvio_closed_forms(oracle_mod):
+    # all tokens pick expert 0 among distinct picks: cnt_0 = T, maxvio = E/K - 1
+    R, S, E, K = 2, 8, 8, 2
+    T = R * S
+    idx = np.stack([np.zeros(T, np.int32), 1 + np.arange(T, dtype=np.int32) % (E - 1)], 1)
+    got = oracle_mod.plan(R, S, E, K, 16, idx)
+    assert got["max_count"] == T
+    assert got["maxvio"] == E / K - 1
+    # every pick forced to one expert: maxvio = E - 1
+    idx = np.full((T, K), 3, np.int32)
+    got = oracle_mod.plan(R, S, E, K, 16, idx)
+    assert got["max_count"] == T * K and got["maxvio"] == E - 1
+
+
+@pytest.mark.parametrize("name,alpha", [("c1", None), ("c2", None), ("c3", 0.0), ("c3", 0.5),
+                                        ("c3", 1.0), ("c3", 1.5)])
+@pytest.mark.parametrize("rule", [0, 1])
+def test_workload_plans_invariants(oracle_mod, name, alpha, rule):
+    cfg = wl.CONFIGS[name]
+    R, S, E, K, B = (cfg[k] for k in ("R", "S", "E", "K", "B"))
+    idx, _ = wl.routing(cfg, seed=0, alpha=alpha)
+    got = oracle_mod.plan(R, S, E, K, B, idx, rule=rule)
+    cnt = np.bincount(idx.reshape(-1), minlength=E)
+    assert got["expert_count"].tolist() == cnt.tolist()
+    assert got["max_count"] == cnt.max()
+    assert got["status"] in (0, 3)
+    if got["status"] == 0:
+        check_plan_invariants(got, idx, R, S, E, K, B, rule)
+    else:
+        assert got["fail_slots"] > B
