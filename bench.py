@@ -1,0 +1,442 @@
+"""Benchmark: one step = plan -> dispatch -> combine over one batch of seeded
+synthetic routing, through the libmoonep C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl moonep|reference]
+                    [--workload c2] [--alpha A] [--rule 0|1] [--sweep FILE]
+
+Prints one JSON line (rank 0).  Timing: W untimed warm-up steps; then K steps,
+each preceded by an L2 flush (a 512 MiB memset, outside the step's events) and
+bracketed by CUDA events on the launching stream; a barrier and a device
+synchronise on both sides of the timed loop; the max over ranks.  value =
+routed (token, k) rows of all ranks / step time.  N > 1 runs N independent
+replicas (each rank its own layer, seed + rank): the path has no exchange step
+on one GPU, so no collective is on the data path.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = ("dispatch+combine GB/s (% of HBM peak) and routed tokens/s vs maxvio; plan µs")
+UNIT = "routed tokens/s"
+FLUSH_BYTES = 512 << 20
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+# ---------------------------------------------------------------- helpers
+def algorithmic_bytes(cfgd):
+    """Bytes each kernel must move (read each input once, write each output
+    once, index traffic included)."""
+    R, S, K, H = cfgd["R"], cfgd["S"], cfgd["K"], cfgd["H"]
+    T, P = R * S, R * S * K
+    fp8 = cfgd.get("payload") == "fp8"
+    row_out = H + (H // 128) * 4 if fp8 else 2 * H
+    return dict(
+        plan=12 * P,
+        dispatch=T * H * 2 + P * row_out + 4 * P,
+        combine=P * H * 2 + T * H * 2 + 8 * P,
+    )
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_hash(name):
+    src = os.path.join(ROOT, "dispatch_moonep_plan_b200", "csrc", name)
+    return hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+
+
+def profiled_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the kernel source as it is now; else None."""
+    if not os.path.exists(PROFILE_TRAFFIC):
+        return None
+    d = json.load(open(PROFILE_TRAFFIC)).get("%s/%s" % (kernel, workload))
+    if not d or d.get("source_sha") != kernel_source_hash(d["source"]):
+        return None
+    return d["dram_bytes_per_launch"]
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index, period=0.005):
+        self.index, self.period = index, period
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def reduce_max(values, world):
+    """Max over ranks of a list of floats (host plumbing for the timing)."""
+    if world == 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor(values, dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.cpu().tolist()
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def rank_seed(base, rank):
+    return base + 1000 * rank
+
+
+# ---------------------------------------------------------------- oracle arm
+def oracle_step_estimate(cfgd, idx, w, x_bits, rule, n_tokens, rng_seed=0):
+    """One oracle step: the full plan, then dispatch + stand-in expert +
+    combine for n sampled tokens, extrapolated to all T tokens.  Returns
+    (seconds for a full step, plan seconds, sample seconds)."""
+    import numpy as np
+
+    import oracle
+    R, S, E, K, B = (cfgd[k] for k in ("R", "S", "E", "K", "B"))
+    T = R * S
+    t0 = time.perf_counter()
+    pl = oracle.plan(R, S, E, K, B, idx, rule=rule)
+    t1 = time.perf_counter()
+    tokens = np.random.default_rng(rng_seed).choice(T, size=min(n_tokens, T), replace=False)
+    oracle.path_tokens(cfgd, x_bits, w, pl, tokens, expert="identity",
+                       payload=cfgd.get("payload", "bf16"))
+    t2 = time.perf_counter()
+    full = (t1 - t0) + (t2 - t1) * T / len(tokens)
+    return full, t1 - t0, t2 - t1
+
+
+def run_reference(args, cfgd):
+    """The CPU oracle as the reference arm (rank 0 only)."""
+    import numpy as np
+
+    from dispatch_moonep_plan_b200 import workloads as wl
+    world, rank, _ = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0
+    if rank != 0:
+        return
+    import oracle
+    oracle.lib()
+    T, P = cfgd["R"] * cfgd["S"], cfgd["R"] * cfgd["S"] * cfgd["K"]
+    idx, w = wl.routing(cfgd, seed=rank_seed(0, 0), alpha=args.alpha)
+    x_bits = wl.bf16_bits(wl.hidden(T, cfgd["H"], seed=0))
+    n_tok = 256
+    for _ in range(args.warmup):
+        oracle_step_estimate(cfgd, idx, w, x_bits, args.rule, n_tok)
+    steps = []
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        steps.append(oracle_step_estimate(cfgd, idx, w, x_bits, args.rule, n_tok, rng_seed=i)[0])
+    wall = time.perf_counter() - t0
+    step_s = statistics.mean(steps)
+    value = P / step_s
+    sample = ("each step: the full oracle plan over all %d picks, then dispatch + identity "
+              "expert + combine of %d sampled tokens, time extrapolated to all %d tokens"
+              % (P, n_tok, T))
+    line = dict(impl="reference", metric=METRIC, value=value, unit=UNIT, n_gpus=args.gpus,
+                steps=args.steps, warmup=args.warmup, ms_per_step=step_s * 1e3,
+                higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16",
+                data="synthetic", config=workload_config(cfgd, args),
+                cpu_baseline=dict(kind="oracle", value=value, unit=UNIT, cores=1, sample=sample),
+                e2e=dict(value=value, unit=UNIT, h2d_bytes_per_step=0, d2h_bytes_per_step=0),
+                wall_s=wall)
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(cfgd, args):
+    c = dict(workload=cfgd["name"], R=cfgd["R"], S=cfgd["S"], E=cfgd["E"], K=cfgd["K"],
+             B=cfgd["B"], H=cfgd["H"], payload=cfgd.get("payload", "bf16"),
+             routing=cfgd["routing"], rule=args.rule,
+             l2="flushed before every step (512 MiB memset outside the step's events)")
+    if cfgd["routing"] == "zipf":
+        c["alpha"] = args.alpha if args.alpha is not None else cfgd["alpha"]
+    if cfgd["routing"] == "logits":
+        c["sigma"] = cfgd["sigma"]
+    return c
+
+
+# ---------------------------------------------------------------- GPU arm
+def run_gpu(args, cfgd, emit=True):
+    import numpy as np
+    import torch
+
+    from dispatch_moonep_plan_b200 import moonep as me
+    from dispatch_moonep_plan_b200 import workloads as wl
+
+    world, rank, local = dist_setup(args) if emit else (1, 0, torch.cuda.current_device())
+    seed = rank_seed(0, rank)
+    cfg = me.config_from(cfgd, args.rule)
+    s = me.sizes(cfg)
+    T, P, H, K = s.tokens, s.picks, cfg.H, cfg.K
+    fp8 = cfg.payload == me.PAYLOAD_FP8
+    idx_np, w_np = wl.routing(cfgd, seed=seed, alpha=args.alpha)
+    x = wl.hidden(T, H, seed=seed, device="cuda")
+    idx = torch.from_numpy(idx_np).cuda()
+    w = torch.from_numpy(w_np).cuda()
+    bufs = me.PlanBuffers(cfg)
+    if fp8:
+        recv = torch.empty((P, H), dtype=torch.uint8, device="cuda")
+        scale = torch.empty((P, H // 128), dtype=torch.float32, device="cuda")
+        eo = torch.empty((P, H), dtype=torch.bfloat16, device="cuda")
+    else:
+        recv = torch.empty((P, H), dtype=torch.bfloat16, device="cuda")
+        scale = None
+        eo = recv  # identity expert: combine reads the receive buffers in place
+    y = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        me.plan(cfg, idx, bufs, stream)
+        if ev:
+            ev[1].record(stream)
+        me.dispatch(cfg, bufs, x, recv, scale, stream)
+        if ev:
+            ev[2].record(stream)
+        if fp8:
+            me.expert_standin(cfg, bufs, recv, scale, me.EXPERT_IDENTITY, eo, stream)
+        if ev:
+            ev[3].record(stream)
+        me.combine(cfg, bufs, eo, w, y, stream)
+        if ev:
+            ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    st = me.plan_status(bufs, stream)
+    if st[0] != me.STATUS_OK:
+        raise SystemExit("plan failed with status %s (rule %d); try --rule 1" % (st, args.rule))
+    maxvio = float(bufs.maxvio.item())
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    region = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        region[0].record(stream)
+        for i in range(args.steps):
+            flush.zero_()
+            step(evs[i])
+        region[1].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    t_plan = [e[0].elapsed_time(e[1]) for e in evs]
+    t_disp = [e[1].elapsed_time(e[2]) for e in evs]
+    t_comb = [e[3].elapsed_time(e[4]) for e in evs]
+    t_step = [a + b + c for a, b, c in zip(t_plan, t_disp, t_comb)]
+    region_ms = region[0].elapsed_time(region[1])
+    m_plan, m_disp, m_comb, m_step = (statistics.mean(v) for v in (t_plan, t_disp, t_comb, t_step))
+    m_plan, m_disp, m_comb, m_step, region_ms = reduce_max(
+        [m_plan, m_disp, m_comb, m_step, region_ms], world)
+
+    # ---- end to end through the C ABI with host buffers ----
+    x_h = x.cpu().pin_memory()
+    idx_h = idx.cpu().pin_memory()
+    w_h = w.cpu().pin_memory()
+    y_h = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
+    h2d = x_h.numel() * 2 + idx_h.numel() * 4 + w_h.numel() * 4
+    d2h = y_h.numel() * 2
+    e2e_steps = max(3, min(args.steps, 50))
+    for _ in range(2):
+        x.copy_(x_h, non_blocking=True)
+        idx.copy_(idx_h, non_blocking=True)
+        w.copy_(w_h, non_blocking=True)
+        step()
+        y_h.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        x.copy_(x_h, non_blocking=True)
+        idx.copy_(idx_h, non_blocking=True)
+        w.copy_(w_h, non_blocking=True)
+        step()
+        y_h.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = reduce_max([e0.elapsed_time(e1) / e2e_steps], world)[0]
+
+    bytes_ = algorithmic_bytes(cfgd)
+    peak, peak_kind = peaks()
+    disp_gbs = bytes_["dispatch"] / (m_disp * 1e-3) / 1e9
+    comb_gbs = bytes_["combine"] / (m_comb * 1e-3) / 1e9
+    dom = "dispatch" if m_disp >= m_comb else "combine"
+    dom_gbs = disp_gbs if dom == "dispatch" else comb_gbs
+    traffic = profiled_traffic(dom, cfgd["name"])
+    value = world * P / (m_step * 1e-3)
+    out = dict(
+        metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps,
+        warmup=args.warmup, ms_per_step=m_step, higher_is_better=True, scaling="weak",
+        vs_baseline=None, dtype="fp8" if fp8 else "bf16",
+        data="synthetic (seeded routing and N(0,1) hidden states; one independent layer per GPU)",
+        config=workload_config(cfgd, args),
+        roofline=dict(bound="hbm", kernel=dom, achieved=dom_gbs, peak=peak, unit="GB/s",
+                      frac=dom_gbs / peak, traffic=traffic,
+                      algorithmic_bytes=bytes_[dom], peak_kind=peak_kind),
+        plan_us=m_plan * 1e3, dispatch_us=m_disp * 1e3, combine_us=m_comb * 1e3,
+        dispatch_GBps=disp_gbs, combine_GBps=comb_gbs,
+        dispatch_frac=disp_gbs / peak, combine_frac=comb_gbs / peak,
+        maxvio=maxvio, tokens_per_s=world * T / (m_step * 1e-3),
+        region_ms=region_ms,
+        e2e=dict(value=world * P / (e2e_ms * 1e-3), unit=UNIT, h2d_bytes_per_step=h2d,
+                 d2h_bytes_per_step=d2h, ms_per_step=e2e_ms),
+        gpu_launches=(4 if fp8 else 3) * args.steps,
+        clocks=clk.summary(),
+    )
+    if rank == 0 and emit and world == 1 and not args.no_cpu_baseline:
+        cb = cpu_baseline(cfgd, idx_np, w_np, x, args.rule)
+        out["cpu_baseline"] = cb
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return out if rank == 0 else None
+
+
+def cpu_baseline(cfgd, idx, w, x_dev, rule, budget_s=12.0):
+    """The oracle, as it stands, on a bounded sample of the same workload."""
+    from dispatch_moonep_plan_b200 import workloads as wl
+    x_bits = wl.bf16_bits(x_dev)
+    T, P = cfgd["R"] * cfgd["S"], cfgd["R"] * cfgd["S"] * cfgd["K"]
+    n = 256
+    full, tp, ts = oracle_step_estimate(cfgd, idx, w, x_bits, rule, n)
+    # grow the sample to use about budget_s of CPU time
+    per_tok = ts / n
+    n2 = int(max(n, min(T, (budget_s - tp) / max(per_tok, 1e-9))))
+    full, tp, ts = oracle_step_estimate(cfgd, idx, w, x_bits, rule, n2, rng_seed=1)
+    return dict(kind="oracle", value=P / full, unit=UNIT, cores=1,
+                sample="full oracle plan (%d picks, %.3f s) + dispatch/identity expert/combine "
+                       "of %d of %d tokens (%.2f s), extrapolated to the whole step"
+                       % (P, tp, n2, T, ts))
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="moonep", choices=["moonep", "reference"])
+    ap.add_argument("--workload", default="c2")
+    ap.add_argument("--alpha", type=float, default=None)
+    ap.add_argument("--rule", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", default=None,
+                    help="also time every workload / skew and write JSON lines to this file")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    from dispatch_moonep_plan_b200 import workloads as wl
+    cfgd = wl.CONFIGS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, cfgd)
+        return
+    out = run_gpu(args, cfgd)
+    if out is not None:
+        print(json.dumps(out), flush=True)
+    if args.sweep and out is not None:
+        run_sweep(args)
+
+
+def run_sweep(args):
+    """Every workload and skew level, one JSON line each (not the headline)."""
+    import torch
+    from dispatch_moonep_plan_b200 import workloads as wl
+    cases = [("c1", None, 0), ("c2", None, 0)]
+    cases += [("c3", a, r) for a in (0.0, 0.5, 1.0, 1.5) for r in (0, 1)]
+    cases += [("c4", None, 0), ("c4", None, 1), ("c5", None, 0), ("c5", None, 1)]
+    with open(args.sweep, "w") as f:
+        for name, alpha, rule in cases:
+            a = argparse.Namespace(**vars(args))
+            a.alpha, a.rule, a.no_cpu_baseline = alpha, rule, True
+            a.steps = min(args.steps, 50)
+            try:
+                out = run_gpu(a, wl.CONFIGS[name], emit=False)
+            except SystemExit as e:
+                out = dict(workload=name, alpha=alpha, rule=rule, failed=str(e))
+            f.write(json.dumps(out) + "\n")
+            f.flush()
+            torch.cuda.empty_cache()
+
+
+if __name__ == "__main__":
+    main()

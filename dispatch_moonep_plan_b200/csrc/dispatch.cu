@@ -1,0 +1,165 @@
+// dispatch.cu -- zero-copy dispatch: every token row goes straight to the K
+// rows the plan gives it in the ranks' expert-grouped receive buffers ("MoonEP"
+// on moses-y.github.io, "What This Does": no permute step, no copy out of a
+// communication buffer).
+//
+// One warp per token (grid-stride).  Lane k < K holds dst_row[t, k]; the row
+// is read once with 16-byte loads that skip L1 and written K times with
+// 16-byte evict-first stores, U loads in flight per lane.  The fp8 variant
+// quantises each 128-element block once (amax over 16 lanes by shuffles,
+// scale = amax/448, q = e4m3(x * (448/amax)) with round-to-nearest-even and
+// saturation) and writes the same codes and scales to all K rows.
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "internal.cuh"
+
+namespace moonep {
+namespace {
+
+constexpr int THREADS = 256;
+constexpr int WARPS = THREADS / 32;
+
+template <int U>
+__global__ void __launch_bounds__(THREADS) dispatch_bf16_kernel(const uint4* __restrict__ x,
+                                                               uint4* __restrict__ recv,
+                                                               const int32_t* __restrict__ dst_row,
+                                                               const int32_t* __restrict__ status,
+                                                               int T, int K, int H8) {
+    const int P = T * K;
+    if (load_status(status) != MOONEP_STATUS_OK) return;
+    const int lane = threadIdx.x & 31;
+    const long long nw = (long long)gridDim.x * WARPS;
+    for (long long t = (long long)blockIdx.x * WARPS + (threadIdx.x >> 5); t < T; t += nw) {
+        const int myrow = lane < K ? __ldg(dst_row + t * K + lane) : 0;
+        const uint4* src = x + t * H8;
+        for (int c0 = 0; c0 < H8; c0 += 32 * U) {
+            uint4 v[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int c = c0 + u * 32 + lane;
+                if (c < H8) v[u] = ld_stream_v4(src + c);
+            }
+            for (int k = 0; k < K; ++k) {
+                const int row = __shfl_sync(0xffffffffu, myrow, k);
+                if ((unsigned)row >= (unsigned)P) continue;  // range guard
+                uint4* dst = recv + (long long)row * H8;
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int c = c0 + u * 32 + lane;
+                    if (c < H8) st_stream_v4(dst + c, v[u]);
+                }
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
+    // low byte <- a, high byte <- b
+    __nv_fp8x2_storage_t r = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+    return (uint32_t)r;
+}
+
+// H8 = H/8 (a multiple of 16): lanes 0-15 and 16-31 of a 32-chunk step each
+// cover one 128-element block.
+template <int U>
+__global__ void __launch_bounds__(THREADS) dispatch_fp8_kernel(const uint4* __restrict__ x,
+                                                              uint8_t* __restrict__ recv,
+                                                              float* __restrict__ recv_scale,
+                                                              const int32_t* __restrict__ dst_row,
+                                                              const int32_t* __restrict__ status,
+                                                              int T, int K, int H8) {
+    const int P = T * K;
+    if (load_status(status) != MOONEP_STATUS_OK) return;
+    const int lane = threadIdx.x & 31;
+    const long long H = (long long)H8 * 8;
+    const int nblk = H8 / 16;
+    const long long nw = (long long)gridDim.x * WARPS;
+    for (long long t = (long long)blockIdx.x * WARPS + (threadIdx.x >> 5); t < T; t += nw) {
+        const int myrow = lane < K ? __ldg(dst_row + t * K + lane) : 0;
+        const uint4* src = x + t * H8;
+        for (int c0 = 0; c0 < H8; c0 += 32 * U) {
+            uint2 q[U];
+            float sc[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int c = c0 + u * 32 + lane;
+                uint4 v = make_uint4(0, 0, 0, 0);
+                if (c < H8) v = ld_stream_v4(src + c);
+                float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                              bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+                float amax = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+                for (int o = 8; o >= 1; o >>= 1)
+                    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+                if (amax == 0.0f) {
+                    sc[u] = 1.0f;
+                    q[u] = make_uint2(0, 0);
+                } else {
+                    sc[u] = __fdiv_rn(amax, 448.0f);
+                    const float inv = __fdiv_rn(448.0f, amax);
+                    float g[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) g[i] = __fmul_rn(f[i], inv);
+                    q[u].x = e4m3x2(g[0], g[1]) | (e4m3x2(g[2], g[3]) << 16);
+                    q[u].y = e4m3x2(g[4], g[5]) | (e4m3x2(g[6], g[7]) << 16);
+                }
+            }
+            for (int k = 0; k < K; ++k) {
+                const long long row = __shfl_sync(0xffffffffu, myrow, k);
+                if ((unsigned long long)row >= (unsigned long long)P) continue;  // range guard
+                uint8_t* dst = recv + row * H;
+                float* sdst = recv_scale + row * nblk;
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int c = c0 + u * 32 + lane;
+                    if (c < H8) {
+                        st_stream_v2(dst + (long long)c * 8, q[u]);
+                        if ((lane & 15) == 0) sdst[c >> 4] = sc[u];
+                    }
+                }
+            }
+        }
+    }
+}
+
+int grid_for(long long work_warps) {
+    const int sms = device_sm_count();
+    long long want = (work_warps + WARPS - 1) / WARPS;
+    long long cap = (long long)sms * (2048 / THREADS);
+    if (want > cap) want = cap;
+    if (want < 1) want = 1;
+    return (int)want;
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch(const moonep_config& c, const moonep_plan_t& p, const void* x,
+                            void* recv, float* recv_scale, cudaStream_t s) {
+    const int T = c.R * c.S;
+    const int H8 = c.H / 8;
+    const int grid = grid_for(T);
+    if (c.payload == MOONEP_PAYLOAD_BF16) {
+        if (H8 >= 256)
+            dispatch_bf16_kernel<8><<<grid, THREADS, 0, s>>>(
+                (const uint4*)x, (uint4*)recv, p.dst_row, p.status, T, c.K, H8);
+        else
+            dispatch_bf16_kernel<2><<<grid, THREADS, 0, s>>>(
+                (const uint4*)x, (uint4*)recv, p.dst_row, p.status, T, c.K, H8);
+    } else {
+        if (H8 >= 128)
+            dispatch_fp8_kernel<4><<<grid, THREADS, 0, s>>>(
+                (const uint4*)x, (uint8_t*)recv, recv_scale, p.dst_row, p.status, T, c.K, H8);
+        else
+            dispatch_fp8_kernel<1><<<grid, THREADS, 0, s>>>(
+                (const uint4*)x, (uint8_t*)recv, recv_scale, p.dst_row, p.status, T, c.K, H8);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace moonep

@@ -1,0 +1,96 @@
+// internal.cuh -- shared device helpers and launch declarations of libmoonep.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moonep.h"
+
+namespace moonep {
+
+// status block words
+constexpr int ST_STATUS = 0;
+constexpr int ST_FAIL_RANK = 1;
+constexpr int ST_FAIL_SLOTS = 2;
+constexpr int ST_MAX_COUNT = 3;
+constexpr int ST_BARRIER1 = 4;
+constexpr int ST_BARRIER2 = 5;
+constexpr int ST_BAD_FLAG = 6;
+
+constexpr int MAX_GRID = 1024;  // planner blocks; sizes the workspace
+
+// ---- PTX wrappers ---------------------------------------------------------
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p)
+{
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void red_release_add_u32(unsigned* p, unsigned v)
+{
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long globaltimer_ns()
+{
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// 16-byte streaming load that skips L1 (read-once data)
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// 16-byte store with the evict-first (streaming) hint
+__device__ __forceinline__ void st_stream_v4(void* p, uint4 v)
+{
+    asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ void st_stream_v2(void* p, uint2 v)
+{
+    asm volatile("st.global.cs.v2.u32 [%0], {%1,%2};" ::"l"(p), "r"(v.x), "r"(v.y) : "memory");
+}
+
+// Read a status word written by an earlier kernel in stream order (L2 copy).
+__device__ __forceinline__ int load_status(const int32_t* status)
+{
+    return __ldcg(status + ST_STATUS);
+}
+
+// ---- launchers (one per kernel file) ---------------------------------------
+struct PlanLaunch {
+    int R, S, E, K, B, rule;
+    const int32_t* idx;
+    moonep_plan_t plan;
+    unsigned long long wait_ns;
+    int barrier_extra;
+};
+cudaError_t launch_plan(const PlanLaunch& a, cudaStream_t s, const char** why);
+size_t plan_workspace_bytes(int E);
+
+cudaError_t launch_dispatch(const moonep_config& c, const moonep_plan_t& p, const void* x,
+                            void* recv, float* recv_scale, cudaStream_t s);
+cudaError_t launch_combine(const moonep_config& c, const moonep_plan_t& p, const void* eo,
+                           const float* w, void* y, cudaStream_t s);
+cudaError_t launch_expert_standin(const moonep_config& c, const moonep_plan_t& p,
+                                  const void* recv, const float* recv_scale, int mode, void* out,
+                                  cudaStream_t s);
+cudaError_t launch_prefetch(const moonep_config& c, const moonep_plan_t& p,
+                            void* const* views, int elem_bytes, cudaStream_t s);
+cudaError_t launch_grad_reduce(const moonep_config& c, const moonep_plan_t& p,
+                               float* const* views, cudaStream_t s);
+
+int device_sm_count();
+
+}  // namespace moonep

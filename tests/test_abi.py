@@ -1,0 +1,91 @@
+"""The C-ABI library on a machine without a GPU: it builds, loads, exports
+every entry point include/moonep.h declares, computes sizes, and rejects bad
+arguments before touching the device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moonep.h")
+
+
+@pytest.fixture(scope="module")
+def m():
+    from dispatch_moonep_plan_b200 import build
+    build.build()
+    from dispatch_moonep_plan_b200 import moonep
+    return moonep
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\w[\w\s\*]*?\b(moonep_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_what_binding_lists(m):
+    assert _declared() == sorted(m.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(m):
+    out = subprocess.run(["nm", "-D", "--defined-only", m.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\s[TW]\s+(moonep_\w+)$", out, re.M))
+    for name in _declared():
+        assert name in exported, name
+        getattr(m.lib, name)
+
+
+def test_version_and_sizes(m):
+    assert m.lib.moonep_version() == 100
+    cfg = m.config(16, 16384, 128, 8, 8, 4096, Hp=1536, payload=m.PAYLOAD_FP8)
+    s = m.sizes(cfg)
+    T, P, C = 16 * 16384, 16 * 16384 * 8, 16384 * 8
+    assert (s.tokens, s.picks, s.rows_per_rank) == (T, P, C)
+    assert s.recv_bytes == P * 4096 and s.recv_scale_bytes == P * 32 * 4
+    assert s.dispatch_buffer_bytes_per_rank == C * 4096 + C * 32 * 4
+    assert s.weight_row_bytes == 4096 * 1536 * 2
+    assert s.prefetch_pool_bytes_per_rank == 8 * 4096 * 1536 * 2
+    assert s.weights_view_bytes == 136 * 4096 * 1536 * 2
+    assert s.cu_seqlens_bytes == 16 * 136 * 4 and s.slot_expert_bytes == 16 * 8 * 4
+    assert s.status_bytes == m.STATUS_WORDS * 4
+
+
+@pytest.mark.parametrize("bad,msg", [
+    (dict(E=6, R=4), "multiple of R"),
+    (dict(H=100), "multiple of 8"),
+    (dict(payload=1, H=64), "128"),
+    (dict(E=2048, R=2), "MAX_E"),
+    (dict(R=256, E=256), "MAX_R"),
+    (dict(B=65), "MAX_B"),
+    (dict(K=33), "MAX_K"),
+    (dict(S=1 << 28, K=8, R=1), "2\\^31"),
+    (dict(S=0), "positive"),
+    (dict(B=-1), "non-negative"),
+    (dict(rule=2), "rule"),
+])
+def test_config_rejected(m, bad, msg):
+    d = dict(R=2, S=8, E=4, K=2, B=2, H=64, Hp=0, payload=0, rule=0)
+    d.update(bad)
+    cfg = m.Config(**d)
+    with pytest.raises(m.MoonEPError, match=msg):
+        m.sizes(cfg)
+
+
+def test_calls_reject_null_arguments_without_a_device(m):
+    cfg = m.config(2, 8, 4, 2, 2, 64)
+    plan = m.Plan()
+    rc = m.lib.moonep_plan(ctypes.byref(cfg), None, ctypes.byref(plan), None)
+    assert rc == m.ERR_INVALID_ARG and b"NULL" in m.lib.moonep_last_error()
+    rc = m.lib.moonep_dispatch(ctypes.byref(cfg), ctypes.byref(plan), None, None, None, None)
+    assert rc == m.ERR_INVALID_ARG
+    rc = m.lib.moonep_combine(ctypes.byref(cfg), None, None, None, None, None)
+    assert rc == m.ERR_INVALID_ARG
+    rc = m.lib.moonep_plan_status(None, None, None)
+    assert rc == m.ERR_INVALID_ARG
+    rc = m.lib.moonep_weights_destroy(None)
+    assert rc == m.ERR_INVALID_ARG
+    assert m.lib.moonep_set_wait_limit_ns(0) == m.ERR_INVALID_ARG
+    assert m.lib.moonep_debug_set_barrier_extra(-1) == m.ERR_INVALID_ARG

@@ -1,0 +1,134 @@
+"""Edge cases and failure reporting on the GPU, through the C ABI: degenerate
+sizes, ragged rows, the largest E and R the planner takes, failed plans that
+must move no data, a bad expert index, and a device wait that runs out."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from dispatch_moonep_plan_b200 import workloads as wl
+from gpu_helpers import bits16, compare_plans, gpu_path, me
+
+pytestmark = pytest.mark.gpu
+
+
+def _cfg(R, S, E, K, B, H, routing="zipf", alpha=1.0, payload="bf16"):
+    return dict(name="edge", R=R, S=S, E=E, K=K, B=B, H=H, Hp=0, routing=routing,
+                alpha=alpha, payload=payload)
+
+
+def _full_check(cfgd, idx, w, seed=0, rule=0, expert="scale"):
+    x = wl.hidden(cfgd["R"] * cfgd["S"], cfgd["H"], seed=seed).cuda()
+    out = gpu_path(cfgd, idx, w, x, rule=rule, expert=expert)
+    o = oracle.plan(cfgd["R"], cfgd["S"], cfgd["E"], cfgd["K"], cfgd["B"], idx, rule=rule)
+    compare_plans(out["bufs"].host(), o)
+    if o["status"] == 0:
+        T = idx.shape[0]
+        y, _ = oracle.path_tokens(cfgd, bits16(x), w, o, np.arange(T), expert=expert,
+                                  payload=cfgd["payload"])
+        assert np.array_equal(bits16(out["y"]), y)
+    return out, o
+
+
+@pytest.mark.parametrize("shape", [
+    (1, 1, 1, 1, 0, 8),        # one rank, one token, one expert
+    (1, 7, 4, 3, 2, 24),       # single rank: never any overflow
+    (4, 1, 4, 1, 1, 8),        # one token per rank, Er = 1
+    (3, 5, 6, 6, 4, 136),      # K = E: every token picks every expert
+    (2, 33, 8, 2, 3, 264),     # ragged: H/8 = 33 chunks, not a multiple of 32
+    (5, 17, 10, 3, 5, 40),
+])
+def test_degenerate_and_ragged(shape):
+    R, S, E, K, B, H = shape
+    cfgd = _cfg(R, S, E, K, B, H)
+    for seed in range(3):
+        idx, w = wl.routing(cfgd, seed=seed)
+        for rule in (0, 1):
+            _full_check(cfgd, idx, w, seed=seed, rule=rule)
+
+
+def test_largest_E_and_R():
+    cfgd = _cfg(128, 16, 1024, 8, 16, 64, alpha=1.2)
+    idx, w = wl.routing(cfgd, seed=0)
+    for rule in (0, 1):
+        _full_check(cfgd, idx, w, rule=rule, expert="identity")
+
+
+def test_duplicate_picks_and_all_to_one():
+    cfgd = _cfg(4, 64, 8, 4, 8, 16)
+    idx = np.full((256, 4), 5, np.int32)  # every pick on one expert
+    w = np.full((256, 4), 0.25, np.float32)
+    out, o = _full_check(cfgd, idx, w, rule=0)
+    assert o["status"] == 0 and o["maxvio"] == 7.0
+
+
+def test_round_robin_B0_balanced():
+    cfgd = _cfg(4, 32, 16, 4, 0, 32, routing="round_robin")
+    idx, w = wl.routing(cfgd)
+    out, o = _full_check(cfgd, idx, w)
+    assert o["status"] == 0
+
+
+def test_slot_budget_moves_no_data():
+    cfgd = _cfg(4, 64, 16, 2, 0, 64, alpha=2.0)  # B = 0 and skewed: must fail
+    idx, w = wl.routing(cfgd, seed=0)
+    x = wl.hidden(256, 64).cuda()
+    out = gpu_path(cfgd, idx, w, x, expert="scale")
+    g = out["bufs"].host()
+    assert g["status"] == me().STATUS_SLOT_BUDGET
+    o = oracle.plan(4, 64, 16, 2, 0, idx)
+    compare_plans(g, o)
+    assert not bool(out["recv"].any()) and not bool(out["eo"].any()) and not bool(out["y"].any())
+    assert me().plan_status(out["bufs"])[:3] == [3, o["fail_rank"], o["fail_slots"]]
+
+
+def test_bad_index_reported_and_no_data_moved():
+    cfgd = _cfg(2, 8, 4, 2, 2, 16)
+    idx, w = wl.routing(cfgd, seed=0)
+    idx[5, 1] = 4  # == E
+    x = wl.hidden(16, 16).cuda()
+    out = gpu_path(cfgd, idx, w, x)
+    assert me().plan_status(out["bufs"])[0] == me().STATUS_BAD_INDEX
+    assert not bool(out["recv"].any()) and not bool(out["y"].any())
+    idx[5, 1] = -3
+    out = gpu_path(cfgd, idx, w, x)
+    assert me().plan_status(out["bufs"])[0] == me().STATUS_BAD_INDEX
+
+
+def test_wait_that_runs_out_reports_timeout():
+    """The planner's first grid-wide wait is told to expect one block more
+    than exists; it gives up after the (short) wait limit, the plan reports
+    TIMEOUT, downstream kernels do nothing, and the context stays usable."""
+    m = me()
+    cfgd = _cfg(2, 64, 8, 2, 2, 32)
+    idx, w = wl.routing(cfgd, seed=0)
+    x = wl.hidden(128, 32).cuda()
+    m.set_wait_limit_ns(20_000_000)
+    m.debug_set_barrier_extra(1)
+    try:
+        out = gpu_path(cfgd, idx, w, x)
+        assert m.plan_status(out["bufs"])[0] == m.STATUS_TIMEOUT
+        assert not bool(out["recv"].any()) and not bool(out["y"].any())
+    finally:
+        m.debug_set_barrier_extra(0)
+        m.set_wait_limit_ns(1_000_000_000)
+    out, o = _full_check(cfgd, idx, w)
+    assert o["status"] == 0
+
+
+def test_invalid_arguments_rejected_before_launch():
+    m = me()
+    cfg = m.config(2, 8, 4, 2, 2, 100)  # H not a multiple of 8
+    with pytest.raises(m.MoonEPError, match="multiple of 8"):
+        m.sizes(cfg)
+    cfg = m.config(2, 8, 4, 2, 2, 64, payload=m.PAYLOAD_FP8)  # fp8 needs H % 128 == 0
+    with pytest.raises(m.MoonEPError, match="128"):
+        m.sizes(cfg)
+    cfg = m.config(2, 8, 4, 2, 2, 128)
+    bufs = m.PlanBuffers(cfg)
+    x = torch.zeros((16, 128), dtype=torch.bfloat16, device="cuda")
+    recv = torch.zeros((32, 128), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(m.MoonEPError, match="recv_scale"):
+        m.dispatch(cfg, bufs, x, recv, recv_scale=torch.zeros(4, device="cuda"))
+    with pytest.raises(m.MoonEPError, match="aligned"):
+        m.dispatch(cfg, bufs, x.view(-1)[1:], recv)
