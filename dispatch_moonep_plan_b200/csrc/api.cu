@@ -53,17 +53,29 @@ const char* check_config(const moonep_config* c) {
     return nullptr;
 }
 
+// The plan outputs every call reads or writes.  The planner's workspace is
+// checked by moonep_plan alone: no other call touches it.
 const char* check_plan(const moonep_config* c, const moonep_plan_t* p) {
     if (!p) return "plan is NULL";
     if (!p->expert_count || !p->rank_load || !p->cu_seqlens || !p->dst_row || !p->src_of_row ||
-        !p->status || !p->maxvio || !p->workspace)
+        !p->status || !p->maxvio)
         return "a plan pointer is NULL";
     if (c->B > 0 && !p->slot_expert) return "slot_expert is NULL";
+    return nullptr;
+}
+
+const char* check_workspace(const moonep_config* c, const moonep_plan_t* p) {
+    if (!p->workspace) return "workspace is NULL";
     if (p->workspace_bytes < moonep::plan_workspace_bytes(c->E)) return "workspace too small";
     return nullptr;
 }
 
 }  // namespace
+
+namespace moonep {
+unsigned long long current_wait_limit_ns() { return g_wait_ns; }
+int current_barrier_extra() { return g_barrier_extra; }
+}  // namespace moonep
 
 extern "C" {
 
@@ -121,6 +133,7 @@ int moonep_plan(const moonep_config* c, const int32_t* topk_idx, const moonep_pl
     const char* fn = "moonep_plan";
     if (const char* why = check_config(c)) return fail(MOONEP_ERR_INVALID_ARG, fn, why);
     if (const char* why = check_plan(c, plan)) return fail(MOONEP_ERR_INVALID_ARG, fn, why);
+    if (const char* why = check_workspace(c, plan)) return fail(MOONEP_ERR_INVALID_ARG, fn, why);
     if (!topk_idx) return fail(MOONEP_ERR_INVALID_ARG, fn, "topk_idx is NULL");
     moonep::PlanLaunch a;
     a.R = c->R; a.S = c->S; a.E = c->E; a.K = c->K; a.B = c->B; a.rule = c->rule;

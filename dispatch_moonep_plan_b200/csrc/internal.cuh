@@ -92,5 +92,7 @@ cudaError_t launch_grad_reduce(const moonep_config& c, const moonep_plan_t& p,
                                float* const* views, cudaStream_t s);
 
 int device_sm_count();
+unsigned long long current_wait_limit_ns();
+int current_barrier_extra();
 
 }  // namespace moonep

@@ -89,3 +89,16 @@ def test_calls_reject_null_arguments_without_a_device(m):
     assert rc == m.ERR_INVALID_ARG
     assert m.lib.moonep_set_wait_limit_ns(0) == m.ERR_INVALID_ARG
     assert m.lib.moonep_debug_set_barrier_extra(-1) == m.ERR_INVALID_ARG
+
+
+def test_workspace_checked_by_the_planner_only(m):
+    """The planner rejects a missing workspace; calls that never read it
+    (dispatch here) get past the plan checks without one and stop at their
+    own first missing argument."""
+    cfg = m.config(2, 8, 4, 2, 2, 64)
+    fake = 16  # an aligned non-NULL address; nothing is launched
+    plan = m.Plan(fake, fake, fake, fake, fake, fake, fake, fake, None, 0)
+    rc = m.lib.moonep_plan(ctypes.byref(cfg), ctypes.c_void_p(fake), ctypes.byref(plan), None)
+    assert rc == m.ERR_INVALID_ARG and b"workspace" in m.lib.moonep_last_error()
+    rc = m.lib.moonep_dispatch(ctypes.byref(cfg), ctypes.byref(plan), None, None, None, None)
+    assert rc == m.ERR_INVALID_ARG and b"x or recv is NULL" in m.lib.moonep_last_error()
