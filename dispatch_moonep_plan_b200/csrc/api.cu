@@ -75,6 +75,10 @@ const char* check_workspace(const moonep_config* c, const moonep_plan_t* p) {
 namespace moonep {
 unsigned long long current_wait_limit_ns() { return g_wait_ns; }
 int current_barrier_extra() { return g_barrier_extra; }
+int set_last_error(int code, const char* fn, const char* why) {
+    const std::string reason(why);  // why may point into the current message
+    return fail(code, fn, reason.c_str());
+}
 }  // namespace moonep
 
 extern "C" {

@@ -94,5 +94,6 @@ cudaError_t launch_grad_reduce(const moonep_config& c, const moonep_plan_t& p,
 int device_sm_count();
 unsigned long long current_wait_limit_ns();
 int current_barrier_extra();
+int set_last_error(int code, const char* fn, const char* why);  // returns code
 
 }  // namespace moonep

@@ -32,13 +32,14 @@ MAX_R = 128
 MAX_B = 64
 MAX_K = 32
 STATUS_WORDS = 8
+NOALLOC_MAX_E = 512
 
 # every symbol include/moonep.h declares
 EXPORTS = ("moonep_version", "moonep_last_error", "moonep_sizes", "moonep_plan",
            "moonep_dispatch", "moonep_combine", "moonep_prefetch", "moonep_grad_reduce",
            "moonep_expert_standin", "moonep_plan_status", "moonep_weights_create",
            "moonep_weights_destroy", "moonep_set_wait_limit_ns",
-           "moonep_debug_set_barrier_extra")
+           "moonep_debug_set_barrier_extra", "moonep_plan_noalloc")
 
 i32, i64, sz, vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p
 
@@ -97,6 +98,7 @@ def _load():
     L.moonep_weights_destroy.argtypes = [P(Weights)]
     L.moonep_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     L.moonep_debug_set_barrier_extra.argtypes = [i32]
+    L.moonep_plan_noalloc.argtypes = [P(Config), vp, P(Plan), vp]
     return L
 
 
@@ -180,6 +182,13 @@ def plan(cfg, topk_idx, bufs, stream=None):
     """moonep_plan: topk_idx int32 [T, K] device tensor (or pointer)."""
     _check(lib.moonep_plan(ctypes.byref(cfg), _ptr(topk_idx), ctypes.byref(bufs.c),
                            _stream(stream)), "moonep_plan")
+
+
+def plan_noalloc(cfg, topk_idx, bufs, stream=None):
+    """moonep_plan_noalloc: the planner without a caller workspace (the
+    library's static scratch is used; ``bufs.c.workspace`` is ignored)."""
+    _check(lib.moonep_plan_noalloc(ctypes.byref(cfg), _ptr(topk_idx), ctypes.byref(bufs.c),
+                                   _stream(stream)), "moonep_plan_noalloc")
 
 
 def dispatch(cfg, bufs, x, recv, recv_scale=None, stream=None):

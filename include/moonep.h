@@ -253,6 +253,32 @@ int moonep_plan_status(const moonep_plan_t* plan, moonep_stream_t stream, int32_
 int moonep_weights_create(const moonep_config* cfg, int32_t elem_bytes, moonep_weights_t* out);
 int moonep_weights_destroy(moonep_weights_t* w);
 
+/* Allocation-free planner.  The web pages have no counterpart to this call:
+ * it is a convenience of this library for callers that cannot give the
+ * planner a workspace buffer -- a plugin whose host framework owns all device
+ * memory through its own allocator and hands out no scratch, or a serving
+ * loop that reserves every buffer at start-up and must not allocate once it
+ * runs.
+ *
+ * Same inputs, outputs and results as moonep_plan(); the workspace fields of
+ * *plan are ignored.  The planner's scratch is instead a static device array
+ * inside this library, sized for E <= MOONEP_NOALLOC_MAX_E (4 MiB + 2 KiB);
+ * every GPU that loads the library holds it until the process exits.  A
+ * larger E returns MOONEP_ERR_INVALID_ARG.  The call itself allocates
+ * nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current) and caches it; make
+ *    that first call before any stream capture.
+ *  - All calls share the one array, which keeps the last call's contents.
+ *    Nothing in it needs clearing between calls (each call rewrites every
+ *    word it reads; the wait counters live in the plan's status block, which
+ *    each call zeroes), but two calls whose kernels overlap on the GPU (other
+ *    streams, other host threads) race on it and produce wrong plans: order
+ *    them on one stream or synchronise between them. */
+#define MOONEP_NOALLOC_MAX_E 512
+int moonep_plan_noalloc(const moonep_config* cfg, const int32_t* topk_idx,
+                        const moonep_plan_t* plan, moonep_stream_t stream);
+
 /* Bound on every device-side wait, in nanoseconds (default 1e9).  A wait
  * that runs out sets MOONEP_STATUS_TIMEOUT and the kernel returns. */
 int moonep_set_wait_limit_ns(uint64_t ns);
