@@ -2,10 +2,11 @@
 synthetic routing, through the libmoonep C ABI.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl moonep|reference]
-                    [--workload c2] [--alpha A] [--rule 0|1] [--sweep FILE]
+                    [--workload uniform] [--alpha A] [--rule 0|1] [--sweep FILE]
 
 Prints one JSON line (rank 0).  Timing: W untimed warm-up steps; then K steps,
-each preceded by an L2 flush (a 512 MiB memset, outside the step's events) and
+each preceded by an L2 flush (a 512 MiB memset, then a 256 MiB read so that the
+memset's dirty lines leave L2 before the step; both outside the step's events) and
 bracketed by CUDA events on the launching stream; a barrier and a device
 synchronise on both sides of the timed loop; the max over ranks.  value =
 routed (token, k) rows of all ranks / step time.  N > 1 runs N independent
@@ -27,7 +28,9 @@ if ROOT not in sys.path:
 
 METRIC = ("dispatch+combine GB/s (% of HBM peak) and routed tokens/s vs maxvio; plan µs")
 UNIT = "routed tokens/s"
-FLUSH_BYTES = 512 << 20
+FLUSH_BYTES = 512 << 20   # written between steps: larger than the 126 MB L2
+FLUSH_READ_BYTES = 256 << 20  # then read, so the flush's dirty lines are written back
+                              # before the step starts and are not charged to it
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
 
 
@@ -222,7 +225,8 @@ def workload_config(cfgd, args):
     c = dict(workload=cfgd["name"], R=cfgd["R"], S=cfgd["S"], E=cfgd["E"], K=cfgd["K"],
              B=cfgd["B"], H=cfgd["H"], payload=cfgd.get("payload", "bf16"),
              routing=cfgd["routing"], rule=args.rule,
-             l2="flushed before every step (512 MiB memset outside the step's events)")
+             l2="flushed before every step (512 MiB memset + 256 MiB read, outside the "
+                "step's events)")
     if cfgd["routing"] == "zipf":
         c["alpha"] = args.alpha if args.alpha is not None else cfgd["alpha"]
     if cfgd["routing"] == "logits":
@@ -258,8 +262,13 @@ def run_gpu(args, cfgd, emit=True):
         scale = None
         eo = recv  # identity expert: combine reads the receive buffers in place
     y = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush_r = torch.zeros(FLUSH_READ_BYTES // 4, dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
+
+    def flush():
+        flush_w.zero_()
+        flush_r.sum()
 
     def step(ev=None):
         if ev:
@@ -279,7 +288,7 @@ def run_gpu(args, cfgd, emit=True):
             ev[4].record(stream)
 
     for _ in range(args.warmup):
-        flush.zero_()
+        flush()
         step()
     torch.cuda.synchronize()
     st = me.plan_status(bufs, stream)
@@ -294,7 +303,7 @@ def run_gpu(args, cfgd, emit=True):
         torch.cuda.synchronize()
         region[0].record(stream)
         for i in range(args.steps):
-            flush.zero_()
+            flush()
             step(evs[i])
         region[1].record(stream)
         torch.cuda.synchronize()
@@ -396,7 +405,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="moonep", choices=["moonep", "reference"])
-    ap.add_argument("--workload", default="c2")
+    ap.add_argument("--workload", default="uniform")
     ap.add_argument("--alpha", type=float, default=None)
     ap.add_argument("--rule", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -421,9 +430,9 @@ def run_sweep(args):
     """Every workload and skew level, one JSON line each (not the headline)."""
     import torch
     from dispatch_moonep_plan_b200 import workloads as wl
-    cases = [("c1", None, 0), ("c2", None, 0)]
-    cases += [("c3", a, r) for a in (0.0, 0.5, 1.0, 1.5) for r in (0, 1)]
-    cases += [("c4", None, 0), ("c4", None, 1), ("c5", None, 0), ("c5", None, 1)]
+    cases = [("tiny", None, 0), ("uniform", None, 0)]
+    cases += [("zipf", a, r) for a in (0.0, 0.5, 1.0, 1.5) for r in (0, 1)]
+    cases += [("hot", None, 0), ("hot", None, 1), ("fp8", None, 0), ("fp8", None, 1)]
     with open(args.sweep, "w") as f:
         for name, alpha, rule in cases:
             a = argparse.Namespace(**vars(args))

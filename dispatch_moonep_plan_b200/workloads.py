@@ -24,17 +24,17 @@ import numpy as np
 
 # The five workloads: sizes, routing recipe and the stand-in expert.
 CONFIGS = {
-    "c1": dict(name="R4-S256-E16-K2-H128-zipf1.0", R=4, S=256, E=16, K=2, H=128, B=4,
+    "tiny": dict(name="R4-S256-E16-K2-H128-zipf1.0", R=4, S=256, E=16, K=2, H=128, B=4,
                Hp=0, routing="zipf", alpha=1.0, expert="identity", payload="bf16"),
-    "c2": dict(name="R8-S4096-E64-K6-H2048-uniform", R=8, S=4096, E=64, K=6, H=2048, B=8,
+    "uniform": dict(name="R8-S4096-E64-K6-H2048-uniform", R=8, S=4096, E=64, K=6, H=2048, B=8,
                Hp=0, routing="logits", sigma=0.1, expert="scale", payload="bf16"),
-    "c3": dict(name="R8-S4096-E256-K8-H7168-zipf", R=8, S=4096, E=256, K=8, H=7168, B=16,
+    "zipf": dict(name="R8-S4096-E256-K8-H7168-zipf", R=8, S=4096, E=256, K=8, H=7168, B=16,
                Hp=0, routing="zipf", alpha=1.0, alphas=(0.0, 0.5, 1.0, 1.5),
                expert="scale", payload="bf16"),
-    "c4": dict(name="R32-S8192-E384-K8-H7168-hot50", R=32, S=8192, E=384, K=8, H=7168,
+    "hot": dict(name="R32-S8192-E384-K8-H7168-hot50", R=32, S=8192, E=384, K=8, H=7168,
                B=16, Hp=0, routing="hot_half", alpha=1.0, expert="identity",
                payload="bf16"),
-    "c5": dict(name="R16-S16384-E128-K8-H4096-zipf1.2-fp8", R=16, S=16384, E=128, K=8,
+    "fp8": dict(name="R16-S16384-E128-K8-H4096-zipf1.2-fp8", R=16, S=16384, E=128, K=8,
                H=4096, B=8, Hp=1536, routing="zipf", alpha=1.2, expert="identity",
                payload="fp8"),
 }

@@ -6,7 +6,7 @@ import torch
 from dispatch_moonep_plan_b200 import workloads as wl
 
 
-def _small(oracle, name="c1", seed=0, **kw):
+def _small(oracle, name="tiny", seed=0, **kw):
     cfg = wl.cfg_with(name, **kw)
     R, S, E, K, B, H = (cfg[k] for k in ("R", "S", "E", "K", "B", "H"))
     idx, w = wl.routing(cfg, seed=seed)
@@ -59,7 +59,7 @@ def test_quant_row_bounds_and_torch(oracle_mod):
 
 
 def test_fp8_rows_identical_across_copies(oracle_mod):
-    cfg, idx, w, x, pl = _small(oracle_mod, "c1", H=256)
+    cfg, idx, w, x, pl = _small(oracle_mod, "tiny", H=256)
     K = cfg["K"]
     rows = pl["dst_row"].reshape(-1).astype(np.int64)
     q, s = oracle_mod.dispatch_rows_fp8(K, x, pl["src_of_row"], rows)
@@ -70,7 +70,7 @@ def test_fp8_rows_identical_across_copies(oracle_mod):
 
 
 def test_scale_expert_uses_row_group(oracle_mod):
-    cfg, idx, w, x, pl = _small(oracle_mod, "c1")
+    cfg, idx, w, x, pl = _small(oracle_mod, "tiny")
     R, S, E, K, B = (cfg[k] for k in ("R", "S", "E", "K", "B"))
     C = S * K
     P = idx.size
@@ -88,7 +88,7 @@ def test_combine_identity_closed_form(oracle_mod):
     """Identity expert: every row of token t is x[t], so y = bf16(sum_k w_k x).
     The binary32 chain then sits within one bf16 rounding (unit roundoff 2^-8)
     plus K binary32 roundings of the exact sum."""
-    cfg, idx, w, x, pl = _small(oracle_mod, "c1")
+    cfg, idx, w, x, pl = _small(oracle_mod, "tiny")
     T = idx.shape[0]
     y, y64 = oracle_mod.path_tokens(cfg, x, w, pl, np.arange(T), expert="identity")
     xv = oracle_mod.bf16_to_f32(x).astype(np.float64)
@@ -125,7 +125,7 @@ def test_combine_scale_expert_against_routing(oracle_mod):
     """Scale expert through the plan equals the same expert applied straight
     from the routing (torch bf16 rounding), so a wrong gather or a wrong
     group expert shows up."""
-    cfg, idx, w, x, pl = _small(oracle_mod, "c1")
+    cfg, idx, w, x, pl = _small(oracle_mod, "tiny")
     T, K, E = idx.shape[0], cfg["K"], cfg["E"]
     y, y64 = oracle_mod.path_tokens(cfg, x, w, pl, np.arange(T), expert="scale")
     xs = torch.from_numpy(oracle_mod.bf16_to_f32(x))

@@ -152,8 +152,8 @@ def test_maxvio_closed_forms(oracle_mod):
     assert got["max_count"] == T * K and got["maxvio"] == E - 1
 
 
-@pytest.mark.parametrize("name,alpha", [("c1", None), ("c2", None), ("c3", 0.0), ("c3", 0.5),
-                                        ("c3", 1.0), ("c3", 1.5)])
+@pytest.mark.parametrize("name,alpha", [("tiny", None), ("uniform", None), ("zipf", 0.0), ("zipf", 0.5),
+                                        ("zipf", 1.0), ("zipf", 1.5)])
 @pytest.mark.parametrize("rule", [0, 1])
 def test_workload_plans_invariants(oracle_mod, name, alpha, rule):
     cfg = wl.CONFIGS[name]
