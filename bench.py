@@ -415,7 +415,7 @@ def main(argv=None):
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     from dispatch_moonep_plan_b200 import workloads as wl
-    cfgd = wl.CONFIGS[args.workload]
+    cfgd = wl.WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference(args, cfgd)
         return
@@ -439,7 +439,7 @@ def run_sweep(args):
             a.alpha, a.rule, a.no_cpu_baseline = alpha, rule, True
             a.steps = min(args.steps, 50)
             try:
-                out = run_gpu(a, wl.CONFIGS[name], emit=False)
+                out = run_gpu(a, wl.WORKLOADS[name], emit=False)
             except SystemExit as e:
                 out = dict(workload=name, alpha=alpha, rule=rule, failed=str(e))
             f.write(json.dumps(out) + "\n")

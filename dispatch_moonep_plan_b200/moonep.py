@@ -115,7 +115,7 @@ def config(R, S, E, K, B, H, Hp=0, payload=PAYLOAD_BF16, rule=RULE_INDEX_ORDER):
 
 
 def config_from(d, rule=RULE_INDEX_ORDER):
-    """Config from a workload dict (see workloads.CONFIGS)."""
+    """Config from a workload dict (see workloads.WORKLOADS)."""
     payload = PAYLOAD_FP8 if d.get("payload") == "fp8" else PAYLOAD_BF16
     return Config(d["R"], d["S"], d["E"], d["K"], d["B"], d["H"], d.get("Hp", 0), payload, rule)
 

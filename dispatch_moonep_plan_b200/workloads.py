@@ -23,7 +23,7 @@ recipe says otherwise.  Hidden states are N(0,1) rounded to bf16.
 import numpy as np
 
 # The five workloads: sizes, routing recipe and the stand-in expert.
-CONFIGS = {
+WORKLOADS = {
     "tiny": dict(name="R4-S256-E16-K2-H128-zipf1.0", R=4, S=256, E=16, K=2, H=128, B=4,
                Hp=0, routing="zipf", alpha=1.0, expert="identity", payload="bf16"),
     "uniform": dict(name="R8-S4096-E64-K6-H2048-uniform", R=8, S=4096, E=64, K=6, H=2048, B=8,
@@ -41,7 +41,7 @@ CONFIGS = {
 
 
 def cfg_with(base, **kw):
-    c = dict(CONFIGS[base]) if isinstance(base, str) else dict(base)
+    c = dict(WORKLOADS[base]) if isinstance(base, str) else dict(base)
     c.update(kw)
     return c
 

@@ -72,7 +72,7 @@ def test_random_small_configs(rule):
 
 @pytest.mark.parametrize("expert", ["identity", "scale"])
 def test_c1_full(expert):
-    cfgd = wl.CONFIGS["tiny"]
+    cfgd = wl.WORKLOADS["tiny"]
     for seed in range(3):
         idx, w = wl.routing(cfgd, seed=seed)
         x = wl.hidden(cfgd["R"] * cfgd["S"], cfgd["H"], seed=seed).cuda()
@@ -81,7 +81,7 @@ def test_c1_full(expert):
 
 
 def test_c2_full():
-    cfgd = wl.CONFIGS["uniform"]
+    cfgd = wl.WORKLOADS["uniform"]
     idx, w = wl.routing(cfgd, seed=0)
     x = wl.hidden(cfgd["R"] * cfgd["S"], cfgd["H"], seed=0).cuda()
     out, o = _check_full_small(cfgd, idx, w, x, 0, "scale")
@@ -153,7 +153,7 @@ def _path_tokens_rows(cfgd, x_rows, w_rows, o, tokens, src_c, expert, payload):
 @pytest.mark.parametrize("alpha", [0.0, 0.5, 1.0, 1.5])
 @pytest.mark.parametrize("rule", [0, 1])
 def test_c3_zipf_sweep(alpha, rule):
-    cfgd = wl.CONFIGS["zipf"]
+    cfgd = wl.WORKLOADS["zipf"]
     idx, w, x = routing_and_x(cfgd, seed=0, alpha=alpha)
     out, o = _check_large(cfgd, idx, w, x, rule, "scale")
     if rule == 1:
@@ -161,7 +161,7 @@ def test_c3_zipf_sweep(alpha, rule):
 
 
 def test_c4_adversarial():
-    cfgd = wl.CONFIGS["hot"]
+    cfgd = wl.WORKLOADS["hot"]
     idx, w, x = routing_and_x(cfgd, seed=0)
     out, o = _check_large(cfgd, idx, w, x, 0, "identity", n_sample=256)
     assert o["status"] == 0
@@ -171,7 +171,7 @@ def test_c4_adversarial():
 
 
 def test_c5_fp8():
-    cfgd = wl.CONFIGS["fp8"]
+    cfgd = wl.WORKLOADS["fp8"]
     idx, w, x = routing_and_x(cfgd, seed=0)
     out, o = _check_large(cfgd, idx, w, x, 0, "identity", n_sample=256)
     assert o["status"] == 0
@@ -194,7 +194,7 @@ def test_c5_fp8():
 
 
 def test_determinism_zipf():
-    cfgd = wl.CONFIGS["zipf"]
+    cfgd = wl.WORKLOADS["zipf"]
     idx, w, x = routing_and_x(cfgd, seed=1, alpha=0.5)
     a = gpu_path(cfgd, idx, w, x, rule=1, expert="scale")
     ha = a["bufs"].host()

@@ -45,7 +45,7 @@ def test_views_alias_home_rows():
 @pytest.mark.parametrize("full", [False, True])
 def test_prefetch_and_grad_reduce(full):
     m = me()
-    cfgd = wl.CONFIGS["fp8"] if full else wl.cfg_with("fp8", R=4, S=512, E=16, B=4, H=1024,
+    cfgd = wl.WORKLOADS["fp8"] if full else wl.cfg_with("fp8", R=4, S=512, E=16, B=4, H=1024,
                                                        Hp=1024, alpha=1.5)
     cfg, bufs, o = _plan(cfgd)
     R, E, B, H, Hp = cfg.R, cfg.E, cfg.B, cfg.H, cfg.Hp

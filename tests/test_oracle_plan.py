@@ -156,7 +156,7 @@ def test_maxvio_closed_forms(oracle_mod):
                                         ("zipf", 1.0), ("zipf", 1.5)])
 @pytest.mark.parametrize("rule", [0, 1])
 def test_workload_plans_invariants(oracle_mod, name, alpha, rule):
-    cfg = wl.CONFIGS[name]
+    cfg = wl.WORKLOADS[name]
     R, S, E, K, B = (cfg[k] for k in ("R", "S", "E", "K", "B"))
     idx, _ = wl.routing(cfg, seed=0, alpha=alpha)
     got = oracle_mod.plan(R, S, E, K, B, idx, rule=rule)

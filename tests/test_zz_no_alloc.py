@@ -54,13 +54,13 @@ def test_noalloc_matches_plan_on_consecutive_calls():
     # first call: a large E (256) leaves its tables in the shared array;
     # the second call, with a smaller E (64) and another routing, must not be
     # affected by them; a third call fails the slot budget like moonep_plan
-    r1, g1 = _plan_both(m, wl.CONFIGS["zipf"], seed=3, rule=1, alpha=1.0)
+    r1, g1 = _plan_both(m, wl.WORKLOADS["zipf"], seed=3, rule=1, alpha=1.0)
     _same(r1, g1)
     assert r1["status"] == 0
-    r2, g2 = _plan_both(m, wl.CONFIGS["uniform"], seed=4, rule=0)
+    r2, g2 = _plan_both(m, wl.WORKLOADS["uniform"], seed=4, rule=0)
     _same(r2, g2)
     assert r2["status"] == 0
-    r3, g3 = _plan_both(m, wl.CONFIGS["zipf"], seed=0, rule=0, alpha=1.5)
+    r3, g3 = _plan_both(m, wl.WORKLOADS["zipf"], seed=0, rule=0, alpha=1.5)
     _same(r3, g3)
     assert r3["status"] == m.STATUS_SLOT_BUDGET
 
