@@ -66,6 +66,7 @@ const char* check_plan(const moonep_config* c, const moonep_plan_t* p) {
 
 const char* check_workspace(const moonep_config* c, const moonep_plan_t* p) {
     if (!p->workspace) return "workspace is NULL";
+    if (!aligned16(p->workspace)) return "workspace must be 16-byte aligned";
     if (p->workspace_bytes < moonep::plan_workspace_bytes(c->E)) return "workspace too small";
     return nullptr;
 }

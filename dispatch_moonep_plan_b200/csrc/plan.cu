@@ -10,23 +10,29 @@
 //   every (token, k) pick plus its inverse.
 //
 // Kernel structure (one block per SM, 1024 threads, cooperative launch so
-// that every block is resident and the grid-wide waits cannot deadlock):
-//   A. each warp owns a contiguous run of picks and builds a private
-//      histogram in shared memory (match_any aggregation); the block writes
-//      its column hist[e][block].
-//   -- grid-wide wait 1 --
-//   B. one warp per expert scans its column over the blocks: off[e][block]
-//      (exclusive) and cnt[e] (total).
-//   -- grid-wide wait 2 --
-//   C. every block computes the (small, O(E + R)) balance step itself from
-//      cnt[], so no third wait is needed; block 0 writes the per-layer
-//      outputs and each block writes cu_seqlens / slot_expert of the ranks it
-//      owns; then every warp walks its picks again in (t, k) order and places
-//      them: its running per-expert offsets start at off[e][block] plus the
-//      counts of the block's earlier warps, so the placement is stable and
-//      deterministic without any ordered atomics.
-// Every wait is bounded (globaltimer); a wait that runs out records
-// MOONEP_STATUS_TIMEOUT and the block returns.
+// that every block is resident and the grid-wide wait cannot deadlock):
+//   A. each block owns a contiguous run of picks, each warp a contiguous part
+//      of it; every warp counts its picks per expert in a private shared
+//      histogram (shared atomics: the order of the counts does not matter
+//      here); the block writes its row hist[block][e].
+//   -- one grid-wide wait --
+//   B. every block reads all rows of hist (16-byte loads when E % 4 == 0):
+//      the per-expert totals, and the counts of the blocks before it (its
+//      offsets).
+//   C. every block computes the small O(E + R) balance step itself from the
+//      totals (no further grid-wide wait is needed); block 0 writes the
+//      per-layer outputs, each block writes cu_seqlens / slot_expert of the
+//      ranks it owns; then every warp walks its picks again, 32 at a time, in
+//      (t, k) order; match_any gives each pick its rank among the group's
+//      picks of the same expert.  A warp's running per-expert offsets start at
+//      the block's offset plus the counts of the block's earlier warps, so the
+//      placement is stable and deterministic without ordered atomics.  The
+//      ranking is bound by the warp-shuffle crossbar (match_any, a 32-lane
+//      bitonic sort and a shuffle loop all measure about 2000 cycles per
+//      group of 32 picks at 32 warps per SM); the positions are looked up in
+//      per-expert tables so that the rest of the walk is a few shared loads.
+// The wait is bounded (globaltimer); when it runs out the block records
+// MOONEP_STATUS_TIMEOUT and returns.
 #include <algorithm>
 
 #include "internal.cuh"
@@ -36,11 +42,14 @@ namespace {
 
 constexpr int THREADS = 1024;
 constexpr int NW = THREADS / 32;
-constexpr int UNR = 8;  // picks per lane loaded ahead in the streaming loops
+constexpr int UNR = 8;   // picks per lane loaded ahead in the streaming loops
+constexpr int BUNR = 8;  // histogram rows per thread loaded ahead in phase B
+constexpr int SCAN_N = 4;
 
 struct PlanParams {
     int R, S, E, K, B, rule, Er, C, P;
     int stash;  // 1: the block's picks are kept in shared memory between phases
+    int chunk;  // shared capacity (ints) of the stash
     const int32_t* idx;
     int32_t* expert_count;
     int32_t* rank_load;
@@ -50,21 +59,25 @@ struct PlanParams {
     int32_t* src_of_row;
     int32_t* status;
     double* maxvio;
-    int32_t* hist;  // [E][G]
-    int32_t* off;   // [E][G]
-    int32_t* cnt;   // [E]
+    int32_t* hist;  // [G][E]
     unsigned long long wait_ns;
     int barrier_extra;
 };
 
 struct Smem {
     int* whist;   // [NW][E] per-warp counts, later per-warp running offsets
-    int* cnt;     // [E]
-    int* kk;      // [E] kept rows of each expert on its home rank
-    int* kb;      // [E] first kept row of each expert in its home rank's buffer
-    int* os;      // [E] start of the expert's rows in the overflow stream
-    int* nzr;     // [E+1] number of experts with overflow before e
-    int* nzlist;  // [E] experts with overflow, ascending
+    int* cnt;     // [E]   picks of each expert (all blocks)
+    int* bcnt;    // [E]   picks of each expert in this block
+    int* bpre;    // [E]   picks of each expert in the blocks before this one
+    int* kk;      // [E]   rows of each expert kept on its home rank
+    int* pc;      // [E+1] exclusive prefix of cnt over experts
+    int* pk;      // [E+1] exclusive prefix of kk over experts
+    int* os;      // [E+1] start of each expert's rows in the overflow stream
+    int* nzr;     // [E+1] experts with overflow before e
+    int* nzlist;  // [E]   experts with overflow, ascending
+    int* kbase;   // [E]   destination row of the expert's first kept pick
+    int* rlo;     // [E]   first rank receiving the expert's overflow
+    int* rhi;     // [E]   last rank receiving the expert's overflow
     int* kept;    // [R]
     int* def;     // [R] C - kept
     int* segs;    // [R] start of the rank's segment in the stream
@@ -72,12 +85,13 @@ struct Smem {
     int* nsl;     // [R] slots the rank needs
     int* fe;      // [R] first expert of the rank's segment (-1: none)
     int* rload;   // [R] home rows before balancing
-    int* scratch; // [72]
-    int* idx;     // [chunk] the block's picks (when stashed)
+    int* scratch; // [2*SCAN_N*32 + 8]
+    int* stash;   // [chunk] the block's picks (when stashed)
 };
 
 __host__ __device__ inline size_t smem_ints(int E, int R) {
-    return (size_t)NW * E + 6 * (size_t)E + 1 + 7 * (size_t)R + 72;
+    return (size_t)NW * E + 8 * (size_t)E + 4 * ((size_t)E + 1) + 7 * (size_t)R +
+           2 * SCAN_N * 32 + 8;
 }
 
 __device__ inline Smem carve(int* base, int E, int R) {
@@ -85,11 +99,17 @@ __device__ inline Smem carve(int* base, int E, int R) {
     int* p = base;
     s.whist = p; p += NW * E;
     s.cnt = p; p += E;
+    s.bcnt = p; p += E;
+    s.bpre = p; p += E;
     s.kk = p; p += E;
-    s.kb = p; p += E;
-    s.os = p; p += E;
-    s.nzr = p; p += E + 1;
     s.nzlist = p; p += E;
+    s.pc = p; p += E + 1;
+    s.pk = p; p += E + 1;
+    s.os = p; p += E + 1;
+    s.nzr = p; p += E + 1;
+    s.kbase = p; p += E;
+    s.rlo = p; p += E;
+    s.rhi = p; p += E;
     s.kept = p; p += R;
     s.def = p; p += R;
     s.segs = p; p += R;
@@ -97,8 +117,8 @@ __device__ inline Smem carve(int* base, int E, int R) {
     s.nsl = p; p += R;
     s.fe = p; p += R;
     s.rload = p; p += R;
-    s.scratch = p; p += 72;
-    s.idx = p;
+    s.scratch = p; p += 2 * SCAN_N * 32 + 8;
+    s.stash = p;
     return s;
 }
 
@@ -111,23 +131,33 @@ __device__ __forceinline__ int warp_incl_scan(int x, int lane) {
     return x;
 }
 
-// Exclusive prefix sum of one value per thread over the block.
-__device__ int block_scan_excl(int v, int* scratch, int* total) {
+// Exclusive prefix sums and totals of N values per thread over the block.
+template <int N>
+__device__ void block_scan(const int (&v)[N], int (&excl)[N], int (&tot)[N], int* scratch) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int x = warp_incl_scan(v, lane);
-    if (lane == 31) scratch[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-        int t = lane < NW ? scratch[lane] : 0;
-        t = warp_incl_scan(t, lane);
-        scratch[32 + lane] = t;
+    int x[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i) x[i] = warp_incl_scan(v[i], lane);
+    if (lane == 31) {
+#pragma unroll
+        for (int i = 0; i < N; ++i) scratch[i * 32 + warp] = x[i];
     }
     __syncthreads();
-    int base = warp ? scratch[32 + warp - 1] : 0;
-    int tot = scratch[32 + NW - 1];
+    if (warp == 0) {
+#pragma unroll
+        for (int i = 0; i < N; ++i) {
+            int t = lane < NW ? scratch[i * 32 + lane] : 0;
+            scratch[(N + i) * 32 + lane] = warp_incl_scan(t, lane);
+        }
+    }
     __syncthreads();
-    if (total) *total = tot;
-    return base + x - v;
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+        const int base = warp ? scratch[(N + i) * 32 + warp - 1] : 0;
+        excl[i] = base + x[i] - v[i];
+        tot[i] = scratch[(N + i) * 32 + NW - 1];
+    }
+    __syncthreads();
 }
 
 // First index i in [0, n) with a[i] > v (n if none).
@@ -154,7 +184,6 @@ __device__ bool grid_wait(unsigned* ctr, unsigned target, unsigned long long lim
                 ok = 0;
                 break;
             }
-            __nanosleep(64);
         }
         __threadfence();
         *flag = ok;
@@ -163,96 +192,109 @@ __device__ bool grid_wait(unsigned* ctr, unsigned target, unsigned long long lim
     return *flag != 0;
 }
 
-// The balance step.  Every block runs it on the same cnt[] and reaches the
+// The balance step.  Every block runs it on the same totals and reaches the
 // same result.  Returns the plan status (OK or SLOT_BUDGET).
-__device__ int balance(const PlanParams& p, Smem& s, int* fail_rank, int* fail_slots) {
-    const int tid = threadIdx.x;
+__device__ int balance(const PlanParams& p, Smem& s, int* misc) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int E = p.E, R = p.R, Er = p.Er, C = p.C, B = p.B;
     const bool ve = tid < E;
     const int e = tid;
     const int c = ve ? s.cnt[e] : 0;
     const int first = ve ? (e / Er) * Er : 0;
 
-    // rows of lower-priority experts of the same rank that are kept first
+    // q = rows of the same rank's experts that are kept before expert e
     int q = 0;
     if (p.rule == MOONEP_RULE_INDEX_ORDER) {
-        int pre = block_scan_excl(c, s.scratch, nullptr);
-        if (ve) s.kb[e] = pre;
+        int v1[1] = {c}, ex1[1], t1[1];
+        block_scan<1>(v1, ex1, t1, s.scratch);
+        if (ve) s.pc[e] = ex1[0];
         __syncthreads();
-        if (ve) q = pre - s.kb[first];
-        __syncthreads();
-    } else {
-        if (ve) {
-            for (int i = 0; i < Er; ++i) {
-                int e2 = first + i, c2 = s.cnt[e2];
-                if (c2 < c || (c2 == c && e2 < e)) q += c2;
-            }
+        if (ve) q = ex1[0] - s.pc[first];
+    } else if (ve) {
+        for (int i = 0; i < Er; ++i) {
+            const int e2 = first + i, c2 = s.cnt[e2];
+            if (c2 < c || (c2 == c && e2 < e)) q += c2;
         }
     }
     const long long room = (long long)C - q;
     const int k = ve ? (int)min((long long)c, max(room, 0LL)) : 0;
-    if (ve) s.kk[e] = k;
-
-    // first kept row of each expert in its home rank (index order)
-    int prek = block_scan_excl(k, s.scratch, nullptr);
-    if (ve) s.kb[e] = prek;
-    __syncthreads();
-    int kbv = ve ? prek - s.kb[first] : 0;
-    __syncthreads();
-    if (ve) s.kb[e] = kbv;
-
-    // overflow stream offsets and the list of experts that overflow
     const int o = c - k;
-    int osv = block_scan_excl(o, s.scratch, nullptr);
     const int flag = (ve && o > 0) ? 1 : 0;
-    int nz_tot = 0;
-    int nzv = block_scan_excl(flag, s.scratch, &nz_tot);
+    int v[SCAN_N] = {c, k, o, flag}, ex[SCAN_N], tot[SCAN_N];
+    block_scan<SCAN_N>(v, ex, tot, s.scratch);
     if (ve) {
-        s.os[e] = osv;
-        s.nzr[e] = nzv;
-        if (flag) s.nzlist[nzv] = e;
+        s.kk[e] = k;
+        s.pc[e] = ex[0];
+        s.pk[e] = ex[1];
+        s.os[e] = ex[2];
+        s.nzr[e] = ex[3];
+        if (flag) s.nzlist[ex[3]] = e;
     }
-    if (tid == 0) s.nzr[E] = nz_tot;
+    if (tid == 0) {
+        s.pc[E] = tot[0];
+        s.pk[E] = tot[1];
+        s.os[E] = tot[2];
+        s.nzr[E] = tot[3];
+    }
     __syncthreads();
 
-    // ranks: kept rows, deficits, segments
-    int kept = 0, load = 0;
-    if (tid < R) {
-        for (int i = 0; i < Er; ++i) {
-            kept += s.kk[tid * Er + i];
-            load += s.cnt[tid * Er + i];
+    // ranks: kept rows, deficits, segments, slots -- one warp, 32 ranks a step
+    if (warp == 0) {
+        int carry = 0, fail_r = -1, fail_n = 0;
+        for (int r0 = 0; r0 < R; r0 += 32) {
+            const int r = r0 + lane;
+            const bool vr = r < R;
+            const int kept = vr ? s.pk[(r + 1) * Er] - s.pk[r * Er] : 0;
+            const int load = vr ? s.pc[(r + 1) * Er] - s.pc[r * Er] : 0;
+            const int d = vr ? C - kept : 0;
+            const int incl = warp_incl_scan(d, lane);
+            const int segs = carry + incl - d;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+            int nsl = 0, fe = -1;
+            if (vr && d > 0) {
+                fe = upper_bound(s.os, E, segs) - 1;
+                const int le = upper_bound(s.os, E, segs + d - 1) - 1;
+                nsl = s.nzr[le] - s.nzr[fe] + 1;
+            }
+            if (vr) {
+                s.kept[r] = kept;
+                s.rload[r] = load;
+                s.def[r] = d;
+                s.segs[r] = segs;
+                s.sege[r] = segs + d;
+                s.nsl[r] = nsl;
+                s.fe[r] = fe;
+            }
+            const unsigned over = __ballot_sync(0xffffffffu, vr && nsl > B);
+            if (over && fail_r < 0) {
+                const int l = __ffs(over) - 1;
+                fail_r = r0 + l;
+                fail_n = __shfl_sync(0xffffffffu, nsl, l);
+            }
         }
-    }
-    const int d = tid < R ? C - kept : 0;
-    int segsv = block_scan_excl(d, s.scratch, nullptr);
-    if (tid < R) {
-        s.kept[tid] = kept;
-        s.rload[tid] = load;
-        s.def[tid] = d;
-        s.segs[tid] = segsv;
-        s.sege[tid] = segsv + d;
-        int nsl = 0, fe = -1;
-        if (d > 0) {
-            fe = upper_bound(s.os, E, segsv) - 1;
-            int le = upper_bound(s.os, E, segsv + d - 1) - 1;
-            nsl = s.nzr[le] - s.nzr[fe] + 1;
+        if (lane == 0) {
+            misc[0] = fail_r;
+            misc[1] = fail_n;
         }
-        s.nsl[tid] = nsl;
-        s.fe[tid] = fe;
     }
     __syncthreads();
-    int st = MOONEP_STATUS_OK;
-    *fail_rank = -1;
-    *fail_slots = 0;
-    for (int r = 0; r < R; ++r) {
-        if (s.nsl[r] > B) {
-            st = MOONEP_STATUS_SLOT_BUDGET;
-            *fail_rank = r;
-            *fail_slots = s.nsl[r];
-            break;
-        }
+    return misc[0] >= 0 ? MOONEP_STATUS_SLOT_BUDGET : MOONEP_STATUS_OK;
+}
+
+// Destination row of the pick at position pos among expert e's picks, or -1.
+__device__ __forceinline__ int place(const PlanParams& p, const Smem& s, int e, int pos) {
+    const int k = s.kk[e];
+    if (pos < k) return s.kbase[e] + pos;
+    const int sidx = s.os[e] + pos - k;
+    int lo = s.rlo[e], hi = s.rhi[e] + 1;  // the receiving rank lies in [rlo, rhi]
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (s.sege[mid] <= sidx) lo = mid + 1;
+        else hi = mid;
     }
-    return st;
+    const int rho = lo;
+    if (rho >= p.R) return -1;
+    return rho * p.C + s.kept[rho] + (sidx - s.segs[rho]);
 }
 
 __global__ void __launch_bounds__(THREADS, 1) plan_kernel(PlanParams p) {
@@ -260,6 +302,7 @@ __global__ void __launch_bounds__(THREADS, 1) plan_kernel(PlanParams p) {
     Smem s = carve(smem_raw, p.E, p.R);
     __shared__ int wait_flag;
     __shared__ int max_count;
+    __shared__ int misc[4];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int G = gridDim.x, b = blockIdx.x;
@@ -271,6 +314,10 @@ __global__ void __launch_bounds__(THREADS, 1) plan_kernel(PlanParams p) {
 
     // ---- A: per-warp histograms ----------------------------------------
     for (int i = tid; i < NW * E; i += THREADS) s.whist[i] = 0;
+    for (int i = tid; i < E; i += THREADS) {
+        s.cnt[i] = 0;
+        s.bpre[i] = 0;
+    }
     if (tid == 0) max_count = 0;
     __syncthreads();
     int bad = 0;
@@ -278,22 +325,18 @@ __global__ void __launch_bounds__(THREADS, 1) plan_kernel(PlanParams p) {
         int ev[UNR];
 #pragma unroll
         for (int u = 0; u < UNR; ++u) {
-            long long q = base + u * 32 + lane;
+            const long long q = base + u * 32 + lane;
             ev[u] = q < whi ? __ldg(p.idx + q) : -1;
         }
 #pragma unroll
         for (int u = 0; u < UNR; ++u) {
-            long long q = base + u * 32 + lane;
-            int e = ev[u];
+            const long long q = base + u * 32 + lane;
             if (q < whi) {
-                if (p.stash) s.idx[q - clo] = e;
-                if (e < 0 || e >= E) {
-                    bad = 1;
-                    e = -1;
-                }
+                const int e = ev[u];
+                if (p.stash) s.stash[q - clo] = e;
+                if (e < 0 || e >= E) bad = 1;
+                else atomicAdd(wh + e, 1);
             }
-            unsigned peers = __match_any_sync(0xffffffffu, e);
-            if (e >= 0 && lane == __ffs(peers) - 1) wh[e] += __popc(peers);
         }
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.status + ST_BAD_FLAG, 1);
@@ -301,7 +344,8 @@ __global__ void __launch_bounds__(THREADS, 1) plan_kernel(PlanParams p) {
     for (int e = tid; e < E; e += THREADS) {
         int t = 0;
         for (int w = 0; w < NW; ++w) t += s.whist[w * E + e];
-        p.hist[(long long)e * G + b] = t;
+        s.bcnt[e] = t;
+        p.hist[(long long)b * E + e] = t;
     }
 
     if (!grid_wait(reinterpret_cast<unsigned*>(p.status + ST_BARRIER1),
@@ -309,44 +353,70 @@ __global__ void __launch_bounds__(THREADS, 1) plan_kernel(PlanParams p) {
         if (tid == 0) atomicMax(p.status + ST_STATUS, MOONEP_STATUS_TIMEOUT);
         return;
     }
-
-    // ---- B: column scans over the blocks, one warp per expert -------------
-    {
-        const int gw = b * NW + warp, GW = G * NW;
-        for (int e = gw; e < E; e += GW) {
-            const int32_t* col = p.hist + (long long)e * G;
-            int32_t* ocol = p.off + (long long)e * G;
-            int carry = 0;
-            for (int base = 0; base < G; base += 32) {
-                int i = base + lane;
-                int v = i < G ? __ldcg(col + i) : 0;
-                int x = warp_incl_scan(v, lane);
-                if (i < G) ocol[i] = carry + x - v;
-                carry += __shfl_sync(0xffffffffu, x, 31);
-            }
-            if (lane == 0) p.cnt[e] = carry;
-        }
-    }
-
-    if (!grid_wait(reinterpret_cast<unsigned*>(p.status + ST_BARRIER2), (unsigned)G, p.wait_ns,
-                   &wait_flag)) {
-        if (tid == 0) atomicMax(p.status + ST_STATUS, MOONEP_STATUS_TIMEOUT);
-        return;
-    }
-    if (__ldcg(p.status + ST_BAD_FLAG)) {
+    if (tid == 0) misc[2] = __ldcg(p.status + ST_BAD_FLAG);
+    __syncthreads();
+    if (misc[2]) {
         if (b == 0 && tid == 0) atomicMax(p.status + ST_STATUS, MOONEP_STATUS_BAD_INDEX);
         return;
     }
 
-    // ---- C: balance step (every block), outputs, placement ---------------
-    for (int e = tid; e < E; e += THREADS) {
-        int c = __ldcg(p.cnt + e);
-        s.cnt[e] = c;
-        atomicMax(&max_count, c);
+    // ---- B: totals and this block's offsets from every block's row --------
+    if ((E & 3) == 0) {
+        const int E4 = E >> 2;
+        const int nparts = THREADS / E4;  // >= 4 since E <= THREADS
+        const int part = tid / E4, e4 = tid - part * E4;
+        if (part < nparts) {
+            int4 tot = make_int4(0, 0, 0, 0), pre = make_int4(0, 0, 0, 0);
+            for (int b0 = part; b0 < G; b0 += nparts * BUNR) {
+                int4 v[BUNR];
+#pragma unroll
+                for (int u = 0; u < BUNR; ++u) {
+                    const int bb = b0 + u * nparts;
+                    v[u] = bb < G ? __ldcg(reinterpret_cast<const int4*>(p.hist + (long long)bb * E) + e4)
+                                  : make_int4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int u = 0; u < BUNR; ++u) {
+                    tot.x += v[u].x; tot.y += v[u].y; tot.z += v[u].z; tot.w += v[u].w;
+                    if (b0 + u * nparts < b) {
+                        pre.x += v[u].x; pre.y += v[u].y; pre.z += v[u].z; pre.w += v[u].w;
+                    }
+                }
+            }
+            const int e = 4 * e4;
+            atomicAdd(s.cnt + e, tot.x); atomicAdd(s.cnt + e + 1, tot.y);
+            atomicAdd(s.cnt + e + 2, tot.z); atomicAdd(s.cnt + e + 3, tot.w);
+            atomicAdd(s.bpre + e, pre.x); atomicAdd(s.bpre + e + 1, pre.y);
+            atomicAdd(s.bpre + e + 2, pre.z); atomicAdd(s.bpre + e + 3, pre.w);
+        }
+    } else {
+        const int nparts = THREADS / E;  // >= 1 since E <= THREADS
+        const int part = tid / E, e = tid - part * E;
+        if (part < nparts) {
+            int tot = 0, pre = 0;
+            for (int b0 = part; b0 < G; b0 += nparts * BUNR) {
+                int v[BUNR];
+#pragma unroll
+                for (int u = 0; u < BUNR; ++u) {
+                    const int bb = b0 + u * nparts;
+                    v[u] = bb < G ? __ldcg(p.hist + (long long)bb * E + e) : 0;
+                }
+#pragma unroll
+                for (int u = 0; u < BUNR; ++u) {
+                    tot += v[u];
+                    if (b0 + u * nparts < b) pre += v[u];
+                }
+            }
+            atomicAdd(s.cnt + e, tot);
+            atomicAdd(s.bpre + e, pre);
+        }
     }
     __syncthreads();
-    int fail_rank, fail_slots;
-    const int st = balance(p, s, &fail_rank, &fail_slots);
+    for (int e = tid; e < E; e += THREADS) atomicMax(&max_count, s.cnt[e]);
+    __syncthreads();
+
+    // ---- C: balance step (every block), outputs, placement ---------------
+    const int st = balance(p, s, misc);
 
     if (b == 0) {
         for (int e = tid; e < E; e += THREADS) p.expert_count[e] = s.cnt[e];
@@ -356,23 +426,24 @@ __global__ void __launch_bounds__(THREADS, 1) plan_kernel(PlanParams p) {
             const double tbar = __ddiv_rn((double)P, (double)E);
             p.maxvio[0] = __dsub_rn(__ddiv_rn((double)mx, tbar), 1.0);
             p.status[ST_MAX_COUNT] = mx;
-            p.status[ST_FAIL_RANK] = fail_rank;
-            p.status[ST_FAIL_SLOTS] = fail_slots;
+            p.status[ST_FAIL_RANK] = misc[0];
+            p.status[ST_FAIL_SLOTS] = misc[1];
             atomicMax(p.status + ST_STATUS, st);
         }
     }
     if (st != MOONEP_STATUS_OK) return;
 
-    const int R = p.R, B = p.B, Er = p.Er, C = p.C;
+    const int R = p.R, B = p.B, Er = p.Er;
     for (int r = b; r < R; r += G) {
         const int kept = s.kept[r], d = s.def[r], segs = s.segs[r], sege = s.sege[r];
         const int nsl = s.nsl[r], fe = s.fe[r];
         const int nz0 = fe >= 0 ? s.nzr[fe] : 0;
+        const int rbase = s.pk[r * Er];
         for (int g = tid; g < E + B; g += THREADS) {
             int v;
             if (g < E) {
                 const int h = g / Er;
-                v = h < r ? 0 : (h > r ? kept : s.kb[g] + s.kk[g]);
+                v = h < r ? 0 : (h > r ? kept : s.pk[g] - rbase + s.kk[g]);
             } else {
                 const int j = g - E;
                 if (j < nsl) {
@@ -389,68 +460,76 @@ __global__ void __launch_bounds__(THREADS, 1) plan_kernel(PlanParams p) {
             p.slot_expert[r * B + j] = j < nsl ? s.nzlist[nz0 + j] : -1;
     }
 
-    // per-warp running offsets: block offset + earlier warps' counts
+    // per-warp running offsets: block offset + earlier warps' counts; and the
+    // per-expert placement tables
     for (int e = tid; e < E; e += THREADS) {
-        int run = __ldcg(p.off + (long long)e * G + b);
+        int run = s.bpre[e];
         for (int w = 0; w < NW; ++w) {
-            int t = s.whist[w * E + e];
+            const int t = s.whist[w * E + e];
             s.whist[w * E + e] = run;
             run += t;
         }
+        const int first = (e / Er) * Er;
+        s.kbase[e] = (e / Er) * p.C + (s.pk[e] - s.pk[first]);
+        const int o = s.cnt[e] - s.kk[e];
+        s.rlo[e] = o > 0 ? upper_bound(s.sege, R, s.os[e]) : 0;
+        s.rhi[e] = o > 0 ? upper_bound(s.sege, R, s.os[e] + o - 1) : 0;
     }
     __syncthreads();
 
     const unsigned lt_mask = (1u << lane) - 1u;
+    int internal = 0;
     for (long long base = wlo; base < whi; base += 32 * UNR) {
+        const int nu = (int)min((long long)UNR, (whi - base + 31) / 32);  // warp-uniform
         int ev[UNR];
 #pragma unroll
         for (int u = 0; u < UNR; ++u) {
-            long long q = base + u * 32 + lane;
-            ev[u] = q < whi ? (p.stash ? s.idx[q - clo] : __ldg(p.idx + q)) : -1;
+            const long long q = base + u * 32 + lane;
+            ev[u] = q < whi ? (p.stash ? s.stash[q - clo] : __ldg(p.idx + q)) : -1;
+        }
+        int pos[UNR];
+#pragma unroll
+        for (int u = 0; u < UNR; ++u) {
+            if (u < nu) {
+                const int e = ev[u];
+                const unsigned peers = __match_any_sync(0xffffffffu, e);
+                if (e >= 0) pos[u] = wh[e] + __popc(peers & lt_mask);
+                __syncwarp();
+                if (e >= 0 && lane == __ffs(peers) - 1) wh[e] += __popc(peers);
+                __syncwarp();
+            }
         }
 #pragma unroll
         for (int u = 0; u < UNR; ++u) {
-            const long long q = base + u * 32 + lane;
             const int e = ev[u];
-            const unsigned peers = __match_any_sync(0xffffffffu, e);
-            int pos = 0;
-            if (e >= 0) pos = wh[e] + __popc(peers & lt_mask);
-            __syncwarp();
-            if (e >= 0 && lane == __ffs(peers) - 1) wh[e] += __popc(peers);
-            __syncwarp();
-            if (e >= 0) {
-                const int k = s.kk[e];
-                int dst = -1;
-                if (pos < k) {
-                    dst = (e / Er) * C + s.kb[e] + pos;
-                } else {
-                    const int sidx = s.os[e] + pos - k;
-                    const int rho = upper_bound(s.sege, R, sidx);
-                    if (rho < R) dst = rho * C + s.kept[rho] + (sidx - s.segs[rho]);
-                }
-                if (dst >= 0 && dst < p.P && pos < s.cnt[e]) {
+            if (u < nu && e >= 0) {
+                const long long q = base + u * 32 + lane;
+                const int dst = place(p, s, e, pos[u]);
+                if (dst >= 0 && dst < p.P && pos[u] < s.cnt[e]) {
                     p.dst_row[q] = dst;
                     p.src_of_row[dst] = (int)q;
                 } else {
-                    // never expected: report instead of writing out of range
-                    atomicMax(p.status + ST_STATUS, MOONEP_STATUS_INTERNAL);
+                    internal = 1;  // never expected: report, do not write
                 }
             }
         }
     }
+    if (internal) atomicMax(p.status + ST_STATUS, MOONEP_STATUS_INTERNAL);
 }
 
 struct DevInfo {
     int sms = 0;
     int max_smem_optin = 0;
+    size_t smem_set = 0;  // largest dynamic smem the kernel has been configured for
 };
 
-DevInfo dev_info() {
+DevInfo& dev_info() {
     static thread_local int cached_dev = -1;
     static thread_local DevInfo info;
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev != cached_dev) {
+        info = DevInfo();
         cudaDeviceGetAttribute(&info.sms, cudaDevAttrMultiProcessorCount, dev);
         cudaDeviceGetAttribute(&info.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
         cached_dev = dev;
@@ -468,7 +547,7 @@ size_t plan_workspace_bytes(int E) {
 }
 
 cudaError_t launch_plan(const PlanLaunch& a, cudaStream_t stream, const char** why) {
-    const DevInfo info = dev_info();
+    DevInfo& info = dev_info();
     const int G = std::min(info.sms, MAX_GRID);
     PlanParams p;
     p.R = a.R; p.S = a.S; p.E = a.E; p.K = a.K; p.B = a.B; p.rule = a.rule;
@@ -484,36 +563,37 @@ cudaError_t launch_plan(const PlanLaunch& a, cudaStream_t stream, const char** w
     p.src_of_row = a.plan.src_of_row;
     p.status = a.plan.status;
     p.maxvio = a.plan.maxvio;
-    int32_t* ws = static_cast<int32_t*>(a.plan.workspace);
-    p.hist = ws;
-    p.off = ws + (size_t)a.E * MAX_GRID;
-    p.cnt = ws + 2 * (size_t)a.E * MAX_GRID;
+    p.hist = static_cast<int32_t*>(a.plan.workspace);
     p.wait_ns = a.wait_ns;
     p.barrier_extra = a.barrier_extra;
 
+    // Shared memory: the fixed part, then the pick stash (saves re-reading
+    // the picks from L2 in the walk) if it fits.
     const size_t base_bytes = smem_ints(a.E, a.R) * 4;
     const long long chunk = ((long long)p.P + G - 1) / G;
-    size_t smem = base_bytes;
-    p.stash = 0;
-    if (base_bytes + (size_t)chunk * 4 <= (size_t)info.max_smem_optin - 1024) {
-        p.stash = 1;
-        smem = base_bytes + (size_t)chunk * 4;
-    }
+    const size_t limit = (size_t)info.max_smem_optin - 1024;
+    p.chunk = (int)chunk;
+    p.stash = base_bytes + (size_t)chunk * 4 <= limit;
+    const size_t smem = base_bytes + (size_t)chunk * 4 * p.stash;
     if (smem > (size_t)info.max_smem_optin) {
         *why = "planner shared memory exceeds the device limit (E or R too large)";
         return cudaErrorInvalidValue;
     }
-    cudaError_t err = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)smem);
-    if (err != cudaSuccess) return err;
-    int per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, plan_kernel, THREADS, smem);
-    if (err != cudaSuccess) return err;
-    if (per_sm < 1) {
-        *why = "planner block does not fit on an SM";
-        return cudaErrorInvalidConfiguration;
+    cudaError_t err;
+    if (smem > info.smem_set) {
+        err = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)smem);
+        if (err != cudaSuccess) return err;
+        int per_sm = 0;
+        err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, plan_kernel, THREADS, smem);
+        if (err != cudaSuccess) return err;
+        if (per_sm < 1) {
+            *why = "planner block does not fit on an SM";
+            return cudaErrorInvalidConfiguration;
+        }
+        info.smem_set = smem;
     }
-    // status block: status, fail info, wait counters and the bad-index flag
+    // status block: status, fail info, the wait counter and the bad-index flag
     err = cudaMemsetAsync(a.plan.status, 0, MOONEP_STATUS_WORDS * sizeof(int32_t), stream);
     if (err != cudaSuccess) return err;
     void* args[] = {&p};

@@ -131,8 +131,8 @@ typedef struct moonep_plan_t {
     int32_t* status;       /* [MOONEP_STATUS_WORDS]: [0] status, [1] failing rank,
                               [2] slots it needs, [3] max_e T_e; [4..7] planner-internal */
     double* maxvio;        /* [1]     max_e(T_e / Tbar) - 1, Tbar = P/E */
-    void* workspace;       /* planner scratch of workspace_bytes; read by moonep_plan
-                              only, so the other calls accept NULL here */
+    void* workspace;       /* planner scratch of workspace_bytes, 16-byte aligned; read by
+                              moonep_plan only, so the other calls accept NULL here */
     size_t workspace_bytes;
 } moonep_plan_t;
 
