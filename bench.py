@@ -318,33 +318,10 @@ def run_gpu(args, cfgd, emit=True):
         [m_plan, m_disp, m_comb, m_step, region_ms], world)
 
     # ---- end to end through the C ABI with host buffers ----
-    x_h = x.cpu().pin_memory()
-    idx_h = idx.cpu().pin_memory()
-    w_h = w.cpu().pin_memory()
-    y_h = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
-    h2d = x_h.numel() * 2 + idx_h.numel() * 4 + w_h.numel() * 4
-    d2h = y_h.numel() * 2
-    e2e_steps = max(3, min(args.steps, 50))
-    for _ in range(2):
-        x.copy_(x_h, non_blocking=True)
-        idx.copy_(idx_h, non_blocking=True)
-        w.copy_(w_h, non_blocking=True)
-        step()
-        y_h.copy_(y, non_blocking=True)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        x.copy_(x_h, non_blocking=True)
-        idx.copy_(idx_h, non_blocking=True)
-        w.copy_(w_h, non_blocking=True)
-        step()
-        y_h.copy_(y, non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    e2e_ms = reduce_max([e0.elapsed_time(e1) / e2e_steps], world)[0]
+    if getattr(args, "no_e2e", False):
+        e2e = dict(ms=float("nan"), serial_ms=float("nan"), h2d=0, d2h=0)
+    else:
+        e2e = e2e_pipelined(me, cfg, bufs, x, idx, w, recv, scale, eo, fp8, args, world)
 
     bytes_ = algorithmic_bytes(cfgd)
     peak, peak_kind = peaks()
@@ -368,11 +345,17 @@ def run_gpu(args, cfgd, emit=True):
         dispatch_frac=disp_gbs / peak, combine_frac=comb_gbs / peak,
         maxvio=maxvio, tokens_per_s=world * T / (m_step * 1e-3),
         region_ms=region_ms,
-        e2e=dict(value=world * P / (e2e_ms * 1e-3), unit=UNIT, h2d_bytes_per_step=h2d,
-                 d2h_bytes_per_step=d2h, ms_per_step=e2e_ms),
+        e2e=dict(value=world * P / (e2e["ms"] * 1e-3), unit=UNIT,
+                 h2d_bytes_per_step=e2e["h2d"], d2h_bytes_per_step=e2e["d2h"],
+                 ms_per_step=e2e["ms"], serial_ms_per_step=e2e["serial_ms"],
+                 how="pinned host x/idx/w in and y out every step; the next step's "
+                     "inputs copy in and the previous step's y copies out on two copy "
+                     "streams while the step computes"),
         gpu_launches=(4 if fp8 else 3) * args.steps,
         clocks=clk.summary(),
     )
+    if emit and not args.no_side:
+        out["side"] = measure_side(me, wl, flush, world)
     if rank == 0 and emit and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline(cfgd, idx_np, w_np, x, args.rule)
         out["cpu_baseline"] = cb
@@ -380,6 +363,156 @@ def run_gpu(args, cfgd, emit=True):
         import torch.distributed as dist
         dist.destroy_process_group()
     return out if rank == 0 else None
+
+
+def e2e_pipelined(me, cfg, bufs, x, idx, w, recv, scale, eo, fp8, args, world):
+    """The step through the C ABI from pinned host buffers: every step copies
+    its own x, idx and w in and its y out.  Inputs and outputs are double
+    buffered on the device; H2D of step i+1 and D2H of step i-1 run on two
+    copy streams while step i computes.  Also times the plain serial loop."""
+    import torch
+    T, H, K = x.shape[0], x.shape[1], idx.shape[1]
+    cs = torch.cuda.current_stream()
+    h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
+    x_h = x.cpu().pin_memory()
+    idx_h = idx.cpu().pin_memory()
+    w_h = w.cpu().pin_memory()
+    y_h = [torch.empty((T, H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    xs = [x, torch.empty_like(x)]
+    idxs = [idx, torch.empty_like(idx)]
+    ws = [w, torch.empty_like(w)]
+    ys = [torch.empty((T, H), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    h2d = x_h.numel() * 2 + idx_h.numel() * 4 + w_h.numel() * 4
+    d2h = y_h[0].numel() * 2
+    n = max(4, min(args.steps, 50))
+
+    def compute(sl):
+        me.plan(cfg, idxs[sl], bufs, cs)
+        me.dispatch(cfg, bufs, xs[sl], recv, scale, cs)
+        if fp8:
+            me.expert_standin(cfg, bufs, recv, scale, me.EXPERT_IDENTITY, eo, cs)
+        me.combine(cfg, bufs, eo, ws[sl], ys[sl], cs)
+
+    def copy_in(sl):
+        xs[sl].copy_(x_h, non_blocking=True)
+        idxs[sl].copy_(idx_h, non_blocking=True)
+        ws[sl].copy_(w_h, non_blocking=True)
+
+    def run(steps, timed):
+        ev = lambda: torch.cuda.Event(enable_timing=timed)  # noqa: E731
+        in_ready = [ev(), ev()]
+        in_free = [ev(), ev()]
+        out_ready = [ev(), ev()]
+        out_free = [ev(), ev()]
+        for e_ in in_free + out_free:
+            e_.record(cs)
+        start, end = ev(), ev()
+        start.record(cs)
+        h2d_s.wait_event(start)
+        with torch.cuda.stream(h2d_s):
+            copy_in(0)
+            in_ready[0].record(h2d_s)
+        for i in range(steps):
+            sl = i % 2
+            if i + 1 < steps:
+                nx = (i + 1) % 2
+                h2d_s.wait_event(in_free[nx])
+                with torch.cuda.stream(h2d_s):
+                    copy_in(nx)
+                    in_ready[nx].record(h2d_s)
+            cs.wait_event(in_ready[sl])
+            cs.wait_event(out_free[sl])
+            compute(sl)
+            in_free[sl].record(cs)
+            out_ready[sl].record(cs)
+            d2h_s.wait_event(out_ready[sl])
+            with torch.cuda.stream(d2h_s):
+                y_h[sl].copy_(ys[sl], non_blocking=True)
+                out_free[sl].record(d2h_s)
+        cs.wait_event(out_free[(steps - 1) % 2])
+        cs.wait_event(out_free[(steps - 2) % 2])
+        end.record(cs)
+        torch.cuda.synchronize()
+        return start.elapsed_time(end) / steps if timed else None
+
+    run(3, False)
+    barrier(world)
+    ms = run(n, True)
+    # the plain serial loop, for comparison
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(cs)
+    for _ in range(n):
+        copy_in(0)
+        compute(0)
+        y_h[0].copy_(ys[0], non_blocking=True)
+    e1.record(cs)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms, serial = reduce_max([ms, e0.elapsed_time(e1) / n], world)
+    return dict(ms=ms, serial_ms=serial, h2d=h2d, d2h=d2h)
+
+
+def measure_side(me, wl, flush, world, reps=10):
+    """Replica prefetch (bf16 weights) and replica grad-reduce (fp32 grads) at
+    the fp8 workload's sizes on VMM-aliased [E+B, H, H'] views."""
+    import numpy as np
+    import torch
+    cfgd = wl.WORKLOADS["fp8"]
+    cfg = me.config_from(cfgd, 0)
+    idx, _ = wl.routing(cfgd, seed=0)
+    bufs = me.PlanBuffers(cfg)
+    me.plan(cfg, torch.from_numpy(idx).cuda(), bufs)
+    torch.cuda.synchronize()
+    st = me.plan_status(bufs)
+    if st[0] != me.STATUS_OK:
+        return dict(failed="plan status %s" % st)
+    se = bufs.slot_expert.cpu().numpy()[:cfg.R * cfg.B]
+    used = se[se >= 0]
+    n_used = int(used.size)
+    reps_per_e = np.bincount(used, minlength=cfg.E)
+    E, B, H, Hp = cfg.E, cfg.B, cfg.H, cfg.Hp
+    peak, _ = peaks()
+
+    def timeit(fn):
+        ts = []
+        for i in range(reps + 2):
+            flush()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            if i >= 2:
+                ts.append(a.elapsed_time(b))
+        return reduce_max([statistics.mean(ts)], world)[0]
+
+    out = dict(workload=cfgd["name"] + " H'=%d" % Hp, used_slots=n_used,
+               replicated_experts=int((reps_per_e > 0).sum()))
+    wv = me.WeightViews(cfg, elem_bytes=2)
+    try:
+        v0 = me.weight_view_tensor(wv, 0, cfg, torch.bfloat16)
+        v0[:E].normal_()
+        torch.cuda.synchronize()
+        t = timeit(lambda: me.prefetch(cfg, bufs, wv.ptrs, 2))
+        nbytes = n_used * 2 * H * Hp * 2
+        out.update(prefetch_us=t * 1e3, prefetch_GBps=nbytes / t / 1e6,
+                   prefetch_frac=nbytes / t / 1e6 / peak, prefetch_bytes=nbytes)
+        del v0
+    finally:
+        wv.close()
+    gv = me.WeightViews(cfg, elem_bytes=4)
+    try:
+        for r in range(cfg.R):
+            me.weight_view_tensor(gv, r, cfg, torch.float32)[E if r else 0:].normal_()
+        torch.cuda.synchronize()
+        t = timeit(lambda: me.grad_reduce(cfg, bufs, gv.ptrs))
+        nbytes = int(sum((2 + n) * H * Hp * 4 for n in reps_per_e if n > 0))
+        out.update(grad_reduce_us=t * 1e3, grad_reduce_GBps=nbytes / t / 1e6,
+                   grad_reduce_frac=nbytes / t / 1e6 / peak, grad_reduce_bytes=nbytes)
+    finally:
+        gv.close()
+    torch.cuda.empty_cache()
+    return out
 
 
 def cpu_baseline(cfgd, idx, w, x_dev, rule, budget_s=12.0):
@@ -409,6 +542,8 @@ def main(argv=None):
     ap.add_argument("--alpha", type=float, default=None)
     ap.add_argument("--rule", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-side", action="store_true",
+                    help="skip the replica prefetch / grad-reduce measurement")
     ap.add_argument("--sweep", default=None,
                     help="also time every workload / skew and write JSON lines to this file")
     args = ap.parse_args(argv)
@@ -436,7 +571,7 @@ def run_sweep(args):
     with open(args.sweep, "w") as f:
         for name, alpha, rule in cases:
             a = argparse.Namespace(**vars(args))
-            a.alpha, a.rule, a.no_cpu_baseline = alpha, rule, True
+            a.alpha, a.rule, a.no_cpu_baseline, a.no_side, a.no_e2e = alpha, rule, True, True, True
             a.steps = min(args.steps, 50)
             try:
                 out = run_gpu(a, wl.WORKLOADS[name], emit=False)

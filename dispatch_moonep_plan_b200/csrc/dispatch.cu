@@ -128,10 +128,10 @@ __global__ void __launch_bounds__(THREADS) dispatch_fp8_kernel(const uint4* __re
     }
 }
 
-int grid_for(long long work_warps) {
+int grid_for(long long work_warps, int blocks_per_sm) {
     const int sms = device_sm_count();
     long long want = (work_warps + WARPS - 1) / WARPS;
-    long long cap = (long long)sms * (2048 / THREADS);
+    long long cap = (long long)sms * blocks_per_sm;
     if (want > cap) want = cap;
     if (want < 1) want = 1;
     return (int)want;
@@ -143,15 +143,23 @@ cudaError_t launch_dispatch(const moonep_config& c, const moonep_plan_t& p, cons
                             void* recv, float* recv_scale, cudaStream_t s) {
     const int T = c.R * c.S;
     const int H8 = c.H / 8;
-    const int grid = grid_for(T);
     if (c.payload == MOONEP_PAYLOAD_BF16) {
+        // 16 chunks per lane (16 loads in flight, 2 blocks resident per SM) and
+        // a grid of 32 blocks per SM that the block scheduler balances: measured
+        // 0.96-0.99 of the copy peak, against 0.91-0.92 for 8 chunks per lane
+        // on one resident wave of blocks.
+        const int grid = grid_for(T, 32);
         if (H8 >= 256)
+            dispatch_bf16_kernel<16><<<grid, THREADS, 0, s>>>(
+                (const uint4*)x, (uint4*)recv, p.dst_row, p.status, T, c.K, H8);
+        else if (H8 >= 64)
             dispatch_bf16_kernel<8><<<grid, THREADS, 0, s>>>(
                 (const uint4*)x, (uint4*)recv, p.dst_row, p.status, T, c.K, H8);
         else
             dispatch_bf16_kernel<2><<<grid, THREADS, 0, s>>>(
                 (const uint4*)x, (uint4*)recv, p.dst_row, p.status, T, c.K, H8);
     } else {
+        const int grid = grid_for(T, 2048 / THREADS);
         if (H8 >= 128)
             dispatch_fp8_kernel<4><<<grid, THREADS, 0, s>>>(
                 (const uint4*)x, (uint8_t*)recv, recv_scale, p.dst_row, p.status, T, c.K, H8);
