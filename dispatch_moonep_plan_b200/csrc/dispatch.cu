@@ -6,7 +6,7 @@
 // One warp per token (grid-stride).  Lane k < K holds dst_row[t, k]; the row
 // is read once with 16-byte loads that skip L1 and written K times with
 // 16-byte evict-first stores, U loads in flight per lane.  The fp8 variant
-// quantises each 128-element block once (amax over 16 lanes by shuffles,
+// quantises each 128-element block once (amax over 8 lanes by shuffles,
 // scale = amax/448, q = e4m3(x * (448/amax)) with round-to-nearest-even and
 // saturation) and writes the same codes and scales to all K rows.
 #include <cuda_bf16.h>
@@ -63,8 +63,12 @@ __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
     return (uint32_t)r;
 }
 
-// H8 = H/8 (a multiple of 16): lanes 0-15 and 16-31 of a 32-chunk step each
-// cover one 128-element block.
+// fp8: each lane owns 16 consecutive elements (a "unit", two 16-byte loads);
+// 8 lanes make one 128-element block, so the block amax is 3 xor-shuffles.  A
+// lane's 16 codes leave as one 16-byte store per destination row.  The
+// scales of a row are collected in shared memory (one float per block) and
+// written as one contiguous run per destination row once the row is done.
+// H % 128 == 0, so a row has a whole number of 8-lane blocks.
 template <int U>
 __global__ void __launch_bounds__(THREADS) dispatch_fp8_kernel(const uint4* __restrict__ x,
                                                               uint8_t* __restrict__ recv,
@@ -72,59 +76,73 @@ __global__ void __launch_bounds__(THREADS) dispatch_fp8_kernel(const uint4* __re
                                                               const int32_t* __restrict__ dst_row,
                                                               const int32_t* __restrict__ status,
                                                               int T, int K, int H8) {
-    const int P = T * K;
     if (load_status(status) != MOONEP_STATUS_OK) return;
-    const int lane = threadIdx.x & 31;
+    extern __shared__ float row_scales[];  // [WARPS][H8/16]
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int P = T * K;
     const long long H = (long long)H8 * 8;
+    const int nunits = H8 / 2;
     const int nblk = H8 / 16;
+    float* wsc = row_scales + warp * nblk;
     const long long nw = (long long)gridDim.x * WARPS;
-    for (long long t = (long long)blockIdx.x * WARPS + (threadIdx.x >> 5); t < T; t += nw) {
+    for (long long t = (long long)blockIdx.x * WARPS + warp; t < T; t += nw) {
         const int myrow = lane < K ? __ldg(dst_row + t * K + lane) : 0;
         const uint4* src = x + t * H8;
-        for (int c0 = 0; c0 < H8; c0 += 32 * U) {
-            uint2 q[U];
-            float sc[U];
+        for (int m0 = 0; m0 < nunits; m0 += 32 * U) {
+            uint4 q[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                const int c = c0 + u * 32 + lane;
-                uint4 v = make_uint4(0, 0, 0, 0);
-                if (c < H8) v = ld_stream_v4(src + c);
-                float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
-                              bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+                const int m = m0 + u * 32 + lane;
+                uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
+                if (m < nunits) {
+                    a = ld_stream_v4(src + 2 * m);
+                    b = ld_stream_v4(src + 2 * m + 1);
+                }
+                const float f[16] = {bf16_lo(a.x), bf16_hi(a.x), bf16_lo(a.y), bf16_hi(a.y),
+                                     bf16_lo(a.z), bf16_hi(a.z), bf16_lo(a.w), bf16_hi(a.w),
+                                     bf16_lo(b.x), bf16_hi(b.x), bf16_lo(b.y), bf16_hi(b.y),
+                                     bf16_lo(b.z), bf16_hi(b.z), bf16_lo(b.w), bf16_hi(b.w)};
                 float amax = 0.0f;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+                for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
 #pragma unroll
-                for (int o = 8; o >= 1; o >>= 1)
+                for (int o = 4; o >= 1; o >>= 1)
                     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+                float sc;
                 if (amax == 0.0f) {
-                    sc[u] = 1.0f;
-                    q[u] = make_uint2(0, 0);
+                    sc = 1.0f;
+                    q[u] = make_uint4(0, 0, 0, 0);
                 } else {
-                    sc[u] = __fdiv_rn(amax, 448.0f);
+                    sc = __fdiv_rn(amax, 448.0f);
                     const float inv = __fdiv_rn(448.0f, amax);
-                    float g[8];
+                    float g[16];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) g[i] = __fmul_rn(f[i], inv);
+                    for (int i = 0; i < 16; ++i) g[i] = __fmul_rn(f[i], inv);
                     q[u].x = e4m3x2(g[0], g[1]) | (e4m3x2(g[2], g[3]) << 16);
                     q[u].y = e4m3x2(g[4], g[5]) | (e4m3x2(g[6], g[7]) << 16);
+                    q[u].z = e4m3x2(g[8], g[9]) | (e4m3x2(g[10], g[11]) << 16);
+                    q[u].w = e4m3x2(g[12], g[13]) | (e4m3x2(g[14], g[15]) << 16);
                 }
+                if ((lane & 7) == 0 && m < nunits) wsc[m >> 3] = sc;
             }
             for (int k = 0; k < K; ++k) {
                 const long long row = __shfl_sync(0xffffffffu, myrow, k);
                 if ((unsigned long long)row >= (unsigned long long)P) continue;  // range guard
                 uint8_t* dst = recv + row * H;
-                float* sdst = recv_scale + row * nblk;
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
-                    const int c = c0 + u * 32 + lane;
-                    if (c < H8) {
-                        st_stream_v2(dst + (long long)c * 8, q[u]);
-                        if ((lane & 15) == 0) sdst[c >> 4] = sc[u];
-                    }
+                    const int m = m0 + u * 32 + lane;
+                    if (m < nunits) st_stream_v4(dst + (long long)m * 16, q[u]);
                 }
             }
         }
+        __syncwarp();
+        for (int k = 0; k < K; ++k) {
+            const long long row = __shfl_sync(0xffffffffu, myrow, k);
+            if ((unsigned long long)row >= (unsigned long long)P) continue;
+            for (int j = lane; j < nblk; j += 32) recv_scale[row * nblk + j] = wsc[j];
+        }
+        __syncwarp();
     }
 }
 
@@ -159,13 +177,18 @@ cudaError_t launch_dispatch(const moonep_config& c, const moonep_plan_t& p, cons
             dispatch_bf16_kernel<2><<<grid, THREADS, 0, s>>>(
                 (const uint4*)x, (uint4*)recv, p.dst_row, p.status, T, c.K, H8);
     } else {
-        const int grid = grid_for(T, 2048 / THREADS);
-        if (H8 >= 128)
-            dispatch_fp8_kernel<4><<<grid, THREADS, 0, s>>>(
-                (const uint4*)x, (uint8_t*)recv, recv_scale, p.dst_row, p.status, T, c.K, H8);
-        else
-            dispatch_fp8_kernel<1><<<grid, THREADS, 0, s>>>(
-                (const uint4*)x, (uint8_t*)recv, recv_scale, p.dst_row, p.status, T, c.K, H8);
+        // two units (32 elements, 4 loads) per lane, 32 blocks per SM: 0.92 of
+        // the copy peak against 0.84 for 8 elements per lane with 8-byte stores
+        const int grid = grid_for(T, 32);
+        const size_t smem = (size_t)WARPS * (H8 / 16) * sizeof(float);
+        if (smem > 48 * 1024) {
+            cudaError_t e = cudaFuncSetAttribute(dispatch_fp8_kernel<2>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)smem);
+            if (e != cudaSuccess) return e;
+        }
+        dispatch_fp8_kernel<2><<<grid, THREADS, smem, s>>>(
+            (const uint4*)x, (uint8_t*)recv, recv_scale, p.dst_row, p.status, T, c.K, H8);
     }
     return cudaGetLastError();
 }

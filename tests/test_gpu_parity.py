@@ -205,3 +205,20 @@ def test_determinism_zipf():
     for k in ("dst_row", "src_of_row", "cu_seqlens", "slot_expert"):
         assert np.array_equal(ha[k], hb[k])
     assert torch.equal(ya.view(torch.int16), b["y"].view(torch.int16))
+
+
+@pytest.mark.parametrize("H", [128, 384, 1152, 4224])
+def test_small_fp8_full(H):
+    """fp8 payload element by element: codes, scales, dequantised expert and
+    combine, over several hidden sizes (odd numbers of 128-blocks and of
+    32-lane passes), both rules, identity and scale experts."""
+    rng = np.random.default_rng(H)
+    for it in range(6):
+        cfgd = wl.random_small_cfg(rng, H=H)
+        cfgd["payload"] = "fp8"
+        idx, w = wl.routing(cfgd, seed=it)
+        x = wl.hidden(cfgd["R"] * cfgd["S"], H, seed=it).cuda()
+        if it == 0:
+            x[0].zero_()  # a zero row: scale 1, zero codes
+        for rule in (0, 1):
+            _check_full_small(cfgd, idx, w, x, rule, "scale" if it % 2 else "identity")
