@@ -540,6 +540,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="moonep", choices=["moonep", "reference"])
     ap.add_argument("--workload", default="uniform")
     ap.add_argument("--alpha", type=float, default=None)
+    ap.add_argument("--S", type=int, default=None,
+                    help="tokens per rank, overriding the workload's (for small profiling cases)")
     ap.add_argument("--rule", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-side", action="store_true",
@@ -551,6 +553,9 @@ def main(argv=None):
         ap.error("--warmup must be >= 3")
     from dispatch_moonep_plan_b200 import workloads as wl
     cfgd = wl.WORKLOADS[args.workload]
+    if args.S is not None:
+        cfgd = wl.cfg_with(args.workload, S=args.S, name=cfgd["name"].replace(
+            "S%d" % cfgd["S"], "S%d" % args.S))
     if args.impl == "reference":
         run_reference(args, cfgd)
         return
