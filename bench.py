@@ -355,6 +355,7 @@ def run_gpu(args, cfgd, emit=True):
         clocks=clk.summary(),
     )
     if emit and not args.no_side:
+        out["backward"] = measure_backward(me, cfg, bufs, T, P, H, K, flush, world)
         out["side"] = measure_side(me, wl, flush, world)
     if rank == 0 and emit and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline(cfgd, idx_np, w_np, x, args.rule)
@@ -450,6 +451,44 @@ def e2e_pipelined(me, cfg, bufs, x, idx, w, recv, scale, eo, fp8, args, world):
     barrier(world)
     ms, serial = reduce_max([ms, e0.elapsed_time(e1) / n], world)
     return dict(ms=ms, serial_ms=serial, h2d=h2d, d2h=d2h)
+
+
+def measure_backward(me, cfg, bufs, T, P, H, K, flush, world, reps=10):
+    """Backward of combine (d_expert_out = w * dy per row, d_w = <dy, row>) and
+    of dispatch (dx = sum of the token's K rows) on the bench's workload."""
+    import torch
+    dy = torch.randn((T, H), device="cuda").to(torch.bfloat16)
+    eo = torch.randn((P, H), device="cuda").to(torch.bfloat16)
+    w = torch.rand((T, K), device="cuda")
+    d_eo = torch.empty_like(eo)
+    d_w = torch.empty((T, K), dtype=torch.float32, device="cuda")
+    dx = torch.empty_like(dy)
+    peak, _ = peaks()
+
+    def timeit(fn):
+        ts = []
+        for i in range(reps + 2):
+            flush()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            if i >= 2:
+                ts.append(a.elapsed_time(b))
+        return reduce_max([statistics.mean(ts)], world)[0]
+
+    tc = timeit(lambda: me.combine_backward(cfg, bufs, dy, eo, w, d_eo, d_w))
+    td = timeit(lambda: me.dispatch_backward(cfg, bufs, eo, dx))
+    cb = T * H * 2 + 2 * P * H * 2 + P * 4 + 8 * P
+    db = P * H * 2 + T * H * 2 + 4 * P
+    out = dict(combine_backward_us=tc * 1e3, combine_backward_GBps=cb / tc / 1e6,
+               combine_backward_frac=cb / tc / 1e6 / peak,
+               dispatch_backward_us=td * 1e3, dispatch_backward_GBps=db / td / 1e6,
+               dispatch_backward_frac=db / td / 1e6 / peak)
+    del dy, eo, d_eo, dx
+    torch.cuda.empty_cache()
+    return out
 
 
 def measure_side(me, wl, flush, world, reps=10):

@@ -188,6 +188,36 @@ int moonep_combine(const moonep_config* c, const moonep_plan_t* plan, const void
     return MOONEP_OK;
 }
 
+int moonep_combine_backward(const moonep_config* c, const moonep_plan_t* plan, const void* dy,
+                            const void* expert_out, const float* topk_w, void* d_expert_out,
+                            float* d_topk_w, moonep_stream_t stream) {
+    const char* fn = "moonep_combine_backward";
+    if (const char* why = check_config(c)) return fail(MOONEP_ERR_INVALID_ARG, fn, why);
+    if (const char* why = check_plan(c, plan)) return fail(MOONEP_ERR_INVALID_ARG, fn, why);
+    if (!dy || !expert_out || !topk_w || !d_expert_out || !d_topk_w)
+        return fail(MOONEP_ERR_INVALID_ARG, fn, "a NULL argument");
+    if (!aligned16(dy) || !aligned16(expert_out) || !aligned16(d_expert_out))
+        return fail(MOONEP_ERR_INVALID_ARG, fn, "dy, expert_out and d_expert_out must be 16-byte aligned");
+    cudaError_t e = moonep::launch_combine_backward(*c, *plan, dy, expert_out, topk_w, d_expert_out,
+                                                    d_topk_w, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(fn, e);
+    return MOONEP_OK;
+}
+
+int moonep_dispatch_backward(const moonep_config* c, const moonep_plan_t* plan, const void* d_recv,
+                             void* dx, moonep_stream_t stream) {
+    const char* fn = "moonep_dispatch_backward";
+    if (const char* why = check_config(c)) return fail(MOONEP_ERR_INVALID_ARG, fn, why);
+    if (const char* why = check_plan(c, plan)) return fail(MOONEP_ERR_INVALID_ARG, fn, why);
+    if (!d_recv || !dx) return fail(MOONEP_ERR_INVALID_ARG, fn, "d_recv or dx is NULL");
+    if (!aligned16(d_recv) || !aligned16(dx))
+        return fail(MOONEP_ERR_INVALID_ARG, fn, "d_recv and dx must be 16-byte aligned");
+    cudaError_t e = moonep::launch_dispatch_backward(*c, *plan, d_recv, dx,
+                                                     static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(fn, e);
+    return MOONEP_OK;
+}
+
 int moonep_expert_standin(const moonep_config* c, const moonep_plan_t* plan, const void* recv,
                           const float* recv_scale, int32_t mode, void* out,
                           moonep_stream_t stream) {

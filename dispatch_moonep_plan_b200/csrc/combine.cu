@@ -29,18 +29,27 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
-__device__ __forceinline__ void accum(float* acc, float wk, const uint4& v) {
-    acc[0] = __fmaf_rn(wk, bf16_lo(v.x), acc[0]);
-    acc[1] = __fmaf_rn(wk, bf16_hi(v.x), acc[1]);
-    acc[2] = __fmaf_rn(wk, bf16_lo(v.y), acc[2]);
-    acc[3] = __fmaf_rn(wk, bf16_hi(v.y), acc[3]);
-    acc[4] = __fmaf_rn(wk, bf16_lo(v.z), acc[4]);
-    acc[5] = __fmaf_rn(wk, bf16_hi(v.z), acc[5]);
-    acc[6] = __fmaf_rn(wk, bf16_lo(v.w), acc[6]);
-    acc[7] = __fmaf_rn(wk, bf16_hi(v.w), acc[7]);
+template <bool WEIGHTED>
+__device__ __forceinline__ float step(float acc, float wk, float v) {
+    return WEIGHTED ? __fmaf_rn(wk, v, acc) : __fadd_rn(acc, v);
 }
 
-template <int U>
+template <bool WEIGHTED>
+__device__ __forceinline__ void accum(float* acc, float wk, const uint4& v) {
+    acc[0] = step<WEIGHTED>(acc[0], wk, bf16_lo(v.x));
+    acc[1] = step<WEIGHTED>(acc[1], wk, bf16_hi(v.x));
+    acc[2] = step<WEIGHTED>(acc[2], wk, bf16_lo(v.y));
+    acc[3] = step<WEIGHTED>(acc[3], wk, bf16_hi(v.y));
+    acc[4] = step<WEIGHTED>(acc[4], wk, bf16_lo(v.z));
+    acc[5] = step<WEIGHTED>(acc[5], wk, bf16_hi(v.z));
+    acc[6] = step<WEIGHTED>(acc[6], wk, bf16_lo(v.w));
+    acc[7] = step<WEIGHTED>(acc[7], wk, bf16_hi(v.w));
+}
+
+
+// WEIGHTED = false is the backward of dispatch: dx[t] = bf16(sum_k rows),
+// binary32 additions in k order from zero.
+template <int U, bool WEIGHTED>
 __global__ void __launch_bounds__(THREADS) combine_kernel(const uint4* __restrict__ eo,
                                                          const float* __restrict__ w,
                                                          const int32_t* __restrict__ dst_row,
@@ -53,7 +62,7 @@ __global__ void __launch_bounds__(THREADS) combine_kernel(const uint4* __restric
     for (long long t = (long long)blockIdx.x * WARPS + (threadIdx.x >> 5); t < T; t += nw) {
         int myrow = lane < K ? __ldg(dst_row + t * K + lane) : 0;
         if ((unsigned)myrow >= (unsigned)(T * K)) myrow = 0;  // range guard
-        const float myw = lane < K ? __ldg(w + t * K + lane) : 0.0f;
+        const float myw = (WEIGHTED && lane < K) ? __ldg(w + t * K + lane) : 1.0f;
         for (int c0 = 0; c0 < H8; c0 += 32 * U) {
             float acc[U][8];
 #pragma unroll
@@ -81,7 +90,7 @@ __global__ void __launch_bounds__(THREADS) combine_kernel(const uint4* __restric
                     }
                 }
 #pragma unroll
-                for (int u = 0; u < U; ++u) accum(acc[u], wk, cur[u]);
+                for (int u = 0; u < U; ++u) accum<WEIGHTED>(acc[u], wk, cur[u]);
 #pragma unroll
                 for (int u = 0; u < U; ++u) cur[u] = nxt[u];
             }
@@ -102,7 +111,130 @@ __global__ void __launch_bounds__(THREADS) combine_kernel(const uint4* __restric
     }
 }
 
+// Backward of combine: for each pick, d_eo[row] = bf16(w * float(dy[t])) (one
+// binary32 product), and d_w[t,k] = sum_h dy[t,h] * eo[row,h] in binary32:
+// each lane sums its own elements with an fma chain in a fixed order (its
+// chunks in increasing position, the 8 elements of a chunk in order), then a
+// fixed xor-shuffle tree adds the 32 lane sums, so the result depends only on
+// H, not on the launch.
+template <int U, int KMAX>
+__global__ void __launch_bounds__(THREADS) combine_bwd_kernel(const uint4* __restrict__ dy,
+                                                             const uint4* __restrict__ eo,
+                                                             const float* __restrict__ w,
+                                                             const int32_t* __restrict__ dst_row,
+                                                             uint4* __restrict__ d_eo,
+                                                             float* __restrict__ d_w,
+                                                             const int32_t* __restrict__ status,
+                                                             int T, int K, int H8) {
+    if (load_status(status) != MOONEP_STATUS_OK) return;
+    const int lane = threadIdx.x & 31;
+    const int P = T * K;
+    const long long nw = (long long)gridDim.x * WARPS;
+    for (long long t = (long long)blockIdx.x * WARPS + (threadIdx.x >> 5); t < T; t += nw) {
+        int myrow = lane < K ? __ldg(dst_row + t * K + lane) : 0;
+        if ((unsigned)myrow >= (unsigned)P) myrow = 0;  // range guard
+        const float myw = lane < K ? __ldg(w + t * K + lane) : 0.0f;
+        float part[KMAX];
+#pragma unroll
+        for (int k = 0; k < KMAX; ++k) part[k] = 0.0f;
+        const uint4* g_src = dy + t * H8;
+        for (int c0 = 0; c0 < H8; c0 += 32 * U) {
+            float g[U][8];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int c = c0 + u * 32 + lane;
+                const uint4 v = c < H8 ? ld_stream_v4(g_src + c) : make_uint4(0, 0, 0, 0);
+                g[u][0] = bf16_lo(v.x); g[u][1] = bf16_hi(v.x); g[u][2] = bf16_lo(v.y);
+                g[u][3] = bf16_hi(v.y); g[u][4] = bf16_lo(v.z); g[u][5] = bf16_hi(v.z);
+                g[u][6] = bf16_lo(v.w); g[u][7] = bf16_hi(v.w);
+            }
+#pragma unroll
+            for (int k = 0; k < KMAX; ++k) {
+                if (k < K) {
+                    const long long row = __shfl_sync(0xffffffffu, myrow, k);
+                    const float wk = __shfl_sync(0xffffffffu, myw, k);
+                    const uint4* src = eo + row * H8;
+                    uint4* dst = d_eo + row * H8;
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        const int c = c0 + u * 32 + lane;
+                        if (c < H8) {
+                            const uint4 v = ld_stream_v4(src + c);
+                            const float e[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y),
+                                                bf16_hi(v.y), bf16_lo(v.z), bf16_hi(v.z),
+                                                bf16_lo(v.w), bf16_hi(v.w)};
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) part[k] = __fmaf_rn(g[u][i], e[i], part[k]);
+                            uint4 o;
+                            o.x = pack_bf16x2(__fmul_rn(wk, g[u][0]), __fmul_rn(wk, g[u][1]));
+                            o.y = pack_bf16x2(__fmul_rn(wk, g[u][2]), __fmul_rn(wk, g[u][3]));
+                            o.z = pack_bf16x2(__fmul_rn(wk, g[u][4]), __fmul_rn(wk, g[u][5]));
+                            o.w = pack_bf16x2(__fmul_rn(wk, g[u][6]), __fmul_rn(wk, g[u][7]));
+                            st_stream_v4(dst + c, o);
+                        }
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < KMAX; ++k) {
+            if (k < K) {
+                float v = part[k];
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+                if (lane == 0) d_w[t * K + k] = v;
+            }
+        }
+    }
+}
+
+int grid_4_per_sm(long long T) {
+    const int sms = device_sm_count();
+    long long grid = (T + WARPS - 1) / WARPS;
+    const long long cap = (long long)sms * 4;
+    if (grid > cap) grid = cap;
+    if (grid < 1) grid = 1;
+    return (int)grid;
+}
+
 }  // namespace
+
+cudaError_t launch_dispatch_backward(const moonep_config& c, const moonep_plan_t& p,
+                                     const void* d_recv, void* dx, cudaStream_t s) {
+    const int T = c.R * c.S;
+    const int H8 = c.H / 8;
+    const int grid = grid_4_per_sm(T);
+    if (H8 >= 64)
+        combine_kernel<2, false><<<grid, THREADS, 0, s>>>((const uint4*)d_recv, nullptr, p.dst_row,
+                                                          (uint4*)dx, p.status, T, c.K, H8);
+    else
+        combine_kernel<1, false><<<grid, THREADS, 0, s>>>((const uint4*)d_recv, nullptr, p.dst_row,
+                                                          (uint4*)dx, p.status, T, c.K, H8);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_combine_backward(const moonep_config& c, const moonep_plan_t& p, const void* dy,
+                                    const void* eo, const float* w, void* d_eo, float* d_w,
+                                    cudaStream_t s) {
+    const int T = c.R * c.S;
+    const int H8 = c.H / 8;
+    const int grid = grid_4_per_sm(T);
+    const uint4* dy4 = (const uint4*)dy;
+    const uint4* eo4 = (const uint4*)eo;
+    uint4* de4 = (uint4*)d_eo;
+    if (c.K <= 8) {
+        if (H8 >= 64)
+            combine_bwd_kernel<2, 8><<<grid, THREADS, 0, s>>>(dy4, eo4, w, p.dst_row, de4, d_w,
+                                                             p.status, T, c.K, H8);
+        else
+            combine_bwd_kernel<1, 8><<<grid, THREADS, 0, s>>>(dy4, eo4, w, p.dst_row, de4, d_w,
+                                                             p.status, T, c.K, H8);
+    } else {
+        combine_bwd_kernel<1, MOONEP_MAX_K><<<grid, THREADS, 0, s>>>(dy4, eo4, w, p.dst_row, de4,
+                                                                    d_w, p.status, T, c.K, H8);
+    }
+    return cudaGetLastError();
+}
 
 cudaError_t launch_combine(const moonep_config& c, const moonep_plan_t& p, const void* eo,
                            const float* w, void* y, cudaStream_t s) {
@@ -119,11 +251,11 @@ cudaError_t launch_combine(const moonep_config& c, const moonep_plan_t& p, const
     if (grid > cap) grid = cap;
     if (grid < 1) grid = 1;
     if (H8 >= 64)
-        combine_kernel<2><<<(int)grid, THREADS, 0, s>>>((const uint4*)eo, w, p.dst_row,
-                                                       (uint4*)y, p.status, T, c.K, H8);
+        combine_kernel<2, true><<<(int)grid, THREADS, 0, s>>>((const uint4*)eo, w, p.dst_row,
+                                                             (uint4*)y, p.status, T, c.K, H8);
     else
-        combine_kernel<1><<<(int)grid, THREADS, 0, s>>>((const uint4*)eo, w, p.dst_row,
-                                                       (uint4*)y, p.status, T, c.K, H8);
+        combine_kernel<1, true><<<(int)grid, THREADS, 0, s>>>((const uint4*)eo, w, p.dst_row,
+                                                             (uint4*)y, p.status, T, c.K, H8);
     return cudaGetLastError();
 }
 

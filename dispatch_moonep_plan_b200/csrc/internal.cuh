@@ -83,6 +83,11 @@ cudaError_t launch_dispatch(const moonep_config& c, const moonep_plan_t& p, cons
                             void* recv, float* recv_scale, cudaStream_t s);
 cudaError_t launch_combine(const moonep_config& c, const moonep_plan_t& p, const void* eo,
                            const float* w, void* y, cudaStream_t s);
+cudaError_t launch_dispatch_backward(const moonep_config& c, const moonep_plan_t& p,
+                                     const void* d_recv, void* dx, cudaStream_t s);
+cudaError_t launch_combine_backward(const moonep_config& c, const moonep_plan_t& p, const void* dy,
+                                    const void* eo, const float* w, void* d_eo, float* d_w,
+                                    cudaStream_t s);
 cudaError_t launch_expert_standin(const moonep_config& c, const moonep_plan_t& p,
                                   const void* recv, const float* recv_scale, int mode, void* out,
                                   cudaStream_t s);

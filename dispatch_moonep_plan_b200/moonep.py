@@ -39,7 +39,8 @@ EXPORTS = ("moonep_version", "moonep_last_error", "moonep_sizes", "moonep_plan",
            "moonep_dispatch", "moonep_combine", "moonep_prefetch", "moonep_grad_reduce",
            "moonep_expert_standin", "moonep_plan_status", "moonep_weights_create",
            "moonep_weights_destroy", "moonep_set_wait_limit_ns",
-           "moonep_debug_set_barrier_extra", "moonep_plan_noalloc")
+           "moonep_debug_set_barrier_extra", "moonep_plan_noalloc", "moonep_combine_backward",
+           "moonep_dispatch_backward")
 
 i32, i64, sz, vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p
 
@@ -99,6 +100,8 @@ def _load():
     L.moonep_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     L.moonep_debug_set_barrier_extra.argtypes = [i32]
     L.moonep_plan_noalloc.argtypes = [P(Config), vp, P(Plan), vp]
+    L.moonep_combine_backward.argtypes = [P(Config), P(Plan), vp, vp, vp, vp, vp, vp]
+    L.moonep_dispatch_backward.argtypes = [P(Config), P(Plan), vp, vp, vp]
     return L
 
 
@@ -199,6 +202,17 @@ def dispatch(cfg, bufs, x, recv, recv_scale=None, stream=None):
 def combine(cfg, bufs, expert_out, topk_w, y, stream=None):
     _check(lib.moonep_combine(ctypes.byref(cfg), ctypes.byref(bufs.c), _ptr(expert_out),
                               _ptr(topk_w), _ptr(y), _stream(stream)), "moonep_combine")
+
+
+def combine_backward(cfg, bufs, dy, expert_out, topk_w, d_expert_out, d_topk_w, stream=None):
+    _check(lib.moonep_combine_backward(ctypes.byref(cfg), ctypes.byref(bufs.c), _ptr(dy),
+                                       _ptr(expert_out), _ptr(topk_w), _ptr(d_expert_out),
+                                       _ptr(d_topk_w), _stream(stream)), "moonep_combine_backward")
+
+
+def dispatch_backward(cfg, bufs, d_recv, dx, stream=None):
+    _check(lib.moonep_dispatch_backward(ctypes.byref(cfg), ctypes.byref(bufs.c), _ptr(d_recv),
+                                        _ptr(dx), _stream(stream)), "moonep_dispatch_backward")
 
 
 def expert_standin(cfg, bufs, recv, recv_scale, mode, out, stream=None):

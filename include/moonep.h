@@ -205,6 +205,33 @@ int moonep_dispatch(const moonep_config* cfg, const moonep_plan_t* plan, const v
 int moonep_combine(const moonep_config* cfg, const moonep_plan_t* plan, const void* expert_out,
                    const float* topk_w, void* y, moonep_stream_t stream);
 
+/* Backward of combine, for the layer's backward pass ([blog] "Real-World
+ * Use": the backward pass runs after combine; by the chain rule through
+ * y[t] = sum_k w[t,k] * expert_out[dst_row[t,k]]).
+ *
+ * dy: bf16 [T, H]; expert_out: bf16 [R*C, H] (the forward's expert outputs);
+ * topk_w: fp32 [T, K].  Writes
+ *   d_expert_out bf16 [R*C, H]: row dst_row[t,k] = bf16(w[t,k] * float(dy[t])),
+ *     one binary32 product rounded to nearest even;
+ *   d_topk_w fp32 [T, K]: sum_h float(dy[t,h]) * float(expert_out[row,h]) in
+ *     binary32.  Each of 32 lanes sums its own elements with an fma chain,
+ *     then a fixed shuffle tree adds the lanes, so the result is deterministic
+ *     and within the recursive-summation bound gamma(L+5) * sum|terms| of the
+ *     exact value, L = 8 * ceil(H / 256).
+ * Every row of d_expert_out is written (the rows are a permutation of the
+ * picks). */
+int moonep_combine_backward(const moonep_config* cfg, const moonep_plan_t* plan, const void* dy,
+                            const void* expert_out, const float* topk_w, void* d_expert_out,
+                            float* d_topk_w, moonep_stream_t stream);
+
+/* Backward of dispatch (recv[dst_row[t,k]] = x[t]):
+ * dx[t] = bf16(acc), acc = 0; acc = acc + float(d_recv[dst_row[t,k]]) for
+ * k = 0..K-1, binary32 additions in k order, rounded once to bf16.
+ * d_recv: bf16 [R*C, H] (for the fp8 payload, the gradient with respect to
+ * the dequantised rows); dx: bf16 [T, H]. */
+int moonep_dispatch_backward(const moonep_config* cfg, const moonep_plan_t* plan,
+                             const void* d_recv, void* dx, moonep_stream_t stream);
+
 /* Replica weight prefetch ([ainovat], the paragraph on fetching duplicated
  * experts before expert computation, and the [E+B, H, H'] contract).
  *

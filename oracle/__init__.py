@@ -59,6 +59,8 @@ def lib():
         L.oracle_combine_tokens_f64.argtypes = [ci, ci, cl, f32p, u16p, f64p]
         L.oracle_prefetch.argtypes = [ci, ci, cl, ci, i32p, u8p, u8p]
         L.oracle_grad_reduce.argtypes = [ci, ci, ci, cl, i32p, f32p, f32p]
+        L.oracle_combine_backward_tokens.argtypes = [ci, ci, cl, f32p, u16p, u16p, u16p, f64p]
+        L.oracle_dispatch_backward_tokens.argtypes = [ci, ci, cl, u16p, u16p]
         _lib = L
     return _lib
 
@@ -245,3 +247,27 @@ def path_tokens(cfg, x_bits, w, pl, tokens, expert="identity", payload="bf16"):
     eo = eo.reshape(tokens.size, K, H)
     wt = np.asarray(w, np.float32)[tokens]
     return combine_tokens(wt, eo), combine_tokens_f64(wt, eo)
+
+
+# ---------------------------------------------------------------- backward
+def combine_backward_tokens(w, dy_bits, eo_bits):
+    """w [n,K] fp32, dy [n,H] bf16 bits, eo [n,K,H] bf16 bits ->
+    (d_eo [n,K,H] bf16 bits, d_w [n,K] float64)."""
+    w = _c(w, np.float32)
+    dy_bits = _c(dy_bits, np.uint16)
+    eo_bits = _c(eo_bits, np.uint16)
+    n, K, H = eo_bits.shape
+    d_eo = np.empty((n, K, H), np.uint16)
+    d_w = np.empty((n, K), np.float64)
+    lib().oracle_combine_backward_tokens(K, H, n, w.reshape(-1), dy_bits.reshape(-1),
+                                         eo_bits.reshape(-1), d_eo.reshape(-1), d_w.reshape(-1))
+    return d_eo, d_w
+
+
+def dispatch_backward_tokens(d_recv_bits):
+    """d_recv rows per token [n,K,H] bf16 bits -> dx [n,H] bf16 bits."""
+    d_recv_bits = _c(d_recv_bits, np.uint16)
+    n, K, H = d_recv_bits.shape
+    dx = np.empty((n, H), np.uint16)
+    lib().oracle_dispatch_backward_tokens(K, H, n, d_recv_bits.reshape(-1), dx.reshape(-1))
+    return dx

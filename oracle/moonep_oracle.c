@@ -549,3 +549,50 @@ void oracle_grad_reduce(int R, int B, int E, int64_t elems, const int32_t* slot_
                         d[i] = d[i] + g[i];
                 }
 }
+
+/* ------------------------------------------------------------------ */
+/* Backward of combine and dispatch                                    */
+/* ------------------------------------------------------------------ */
+
+/* The layer's backward pass ([blog] "Real-World Use": the backward reduces
+ * gradients; the chain rule through the two data movements):
+ *  combine  y[t] = sum_k w[t,k] * eo[row(t,k)]  gives
+ *    d_eo[row(t,k)] = bf16(w[t,k] * float(dy[t]))   (one binary32 product,
+ *                                                     rounded once to bf16)
+ *    d_w[t,k]       = sum_h float(dy[t,h]) * float(eo[row(t,k),h])
+ *                     (here in binary64, the exact value up to the final
+ *                      rounding; the GPU's binary32 sum is checked against
+ *                      it within the recursive-summation bound)
+ *  dispatch recv[row(t,k)] = x[t]  gives
+ *    dx[t] = bf16(acc), acc = 0; acc = acc + float(d_recv[row(t,k)]) for
+ *    k = 0..K-1, binary32 additions in k order.
+ * dy, eo rows gathered per requested token: dy [n][H], eo [n][K][H]
+ * (bf16 bits), w [n][K]; outputs d_eo [n][K][H] bf16 bits, d_w [n][K]
+ * (double). */
+void oracle_combine_backward_tokens(int K, int H, int64_t n, const float* w, const uint16_t* dy,
+                                    const uint16_t* eo, uint16_t* d_eo, double* d_w)
+{
+    for (int64_t i = 0; i < n; ++i)
+        for (int k = 0; k < K; ++k) {
+            double dot = 0.0;
+            for (int h = 0; h < H; ++h) {
+                float g = oracle_bf16_to_f32(dy[i * H + h]);
+                float v = oracle_bf16_to_f32(eo[(i * K + k) * H + h]);
+                d_eo[(i * K + k) * H + h] = oracle_bf16_from_f32(w[i * K + k] * g);
+                dot += (double)g * (double)v;
+            }
+            d_w[i * K + k] = dot;
+        }
+}
+
+/* d_recv rows gathered per requested token: [n][K][H] bf16 bits -> dx [n][H]. */
+void oracle_dispatch_backward_tokens(int K, int H, int64_t n, const uint16_t* d_recv, uint16_t* dx)
+{
+    for (int64_t i = 0; i < n; ++i)
+        for (int h = 0; h < H; ++h) {
+            float acc = 0.0f;
+            for (int k = 0; k < K; ++k)
+                acc = acc + oracle_bf16_to_f32(d_recv[(i * K + k) * H + h]);
+            dx[i * H + h] = oracle_bf16_from_f32(acc);
+        }
+}

@@ -170,3 +170,38 @@ def test_grad_reduce_order_and_single_replica(oracle_mod):
     assert np.all(home[2] == 0.0)
     assert np.all(home[0] == np.float32(0.1) + np.float32(0.2))
     assert np.all(home[1] == 0) and np.all(home[3] == 0)
+
+
+def test_combine_backward_against_library(oracle_mod):
+    """d_eo = bf16(w * dy) (torch binary32 product, bf16 cast); d_w is the
+    dot product (numpy binary64)."""
+    rng = np.random.default_rng(21)
+    n, K, H = 40, 6, 72
+    w = rng.random((n, K)).astype(np.float32)
+    dy = oracle_mod.bf16_from_f32(rng.standard_normal((n, H)).astype(np.float32))
+    eo = oracle_mod.bf16_from_f32(rng.standard_normal((n, K, H)).astype(np.float32))
+    d_eo, d_w = oracle_mod.combine_backward_tokens(w, dy, eo)
+    dyf = torch.from_numpy(oracle_mod.bf16_to_f32(dy))
+    ref = (torch.from_numpy(w)[:, :, None] * dyf[:, None, :]).to(torch.bfloat16)
+    assert np.array_equal(d_eo, ref.view(torch.int16).numpy().view(np.uint16))
+    dot = np.einsum("nh,nkh->nk", oracle_mod.bf16_to_f32(dy).astype(np.float64),
+                    oracle_mod.bf16_to_f32(eo).astype(np.float64))
+    assert np.allclose(d_w, dot, rtol=1e-12, atol=1e-12)
+
+
+def test_dispatch_backward_closed_form(oracle_mod):
+    """If every row of token t holds the same bf16 vector v, the binary32 sum
+    of K copies is exact (K <= 8, 8 significant bits), so dx = bf16(K * v)."""
+    rng = np.random.default_rng(22)
+    n, K, H = 30, 8, 40
+    v = oracle_mod.bf16_from_f32(rng.standard_normal((n, H)).astype(np.float32))
+    rows = np.repeat(v[:, None, :], K, axis=1)
+    dx = oracle_mod.dispatch_backward_tokens(rows)
+    ref = torch.from_numpy(oracle_mod.bf16_to_f32(v) * K).to(torch.bfloat16)
+    assert np.array_equal(dx, ref.view(torch.int16).numpy().view(np.uint16))
+    # k order is visible in binary32: (2^24 + 1) - 2^24 + 1 ... with bf16 rows
+    big = oracle_mod.bf16_from_f32(np.array([2.0 ** 24], np.float32))[0]
+    one = oracle_mod.bf16_from_f32(np.array([1.0], np.float32))[0]
+    mbig = oracle_mod.bf16_from_f32(np.array([-(2.0 ** 24)], np.float32))[0]
+    seq = np.array([[[big], [one], [mbig], [one]]], np.uint16)  # ((2^24 + 1) - 2^24) + 1 = 1
+    assert oracle_mod.bf16_to_f32(oracle_mod.dispatch_backward_tokens(seq))[0, 0] == 1.0
