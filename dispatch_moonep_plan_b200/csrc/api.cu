@@ -48,7 +48,8 @@ const char* check_config(const moonep_config* c) {
         return "unknown payload";
     if (c->payload == MOONEP_PAYLOAD_FP8 && c->H % 128 != 0)
         return "fp8 payload needs H to be a multiple of 128";
-    if (c->rule != MOONEP_RULE_INDEX_ORDER && c->rule != MOONEP_RULE_KEEP_LIGHTEST)
+    if (c->rule != MOONEP_RULE_INDEX_ORDER && c->rule != MOONEP_RULE_KEEP_LIGHTEST &&
+        c->rule != MOONEP_RULE_LARGEST_FIRST)
         return "unknown rule";
     return nullptr;
 }

@@ -72,9 +72,12 @@ struct Smem {
     int* kk;      // [E]   rows of each expert kept on its home rank
     int* pc;      // [E+1] exclusive prefix of cnt over experts
     int* pk;      // [E+1] exclusive prefix of kk over experts
-    int* os;      // [E+1] start of each expert's rows in the overflow stream
-    int* nzr;     // [E+1] experts with overflow before e
-    int* nzlist;  // [E]   experts with overflow, ascending
+    int* ov;      // [E]   rows of each expert that overflow its home rank
+    int* item_at; // [E]   the expert at each position of the overflow stream's order
+    int* osi;     // [E+1] start of the stream item at each position (non-decreasing)
+    int* nzri;    // [E+1] items with overflow before each position
+    int* ose;     // [E]   start of each expert's rows in the overflow stream
+    int* nzlist;  // [E]   experts with overflow, in stream order
     int* kbase;   // [E]   destination row of the expert's first kept pick
     int* rlo;     // [E]   first rank receiving the expert's overflow
     int* rhi;     // [E]   last rank receiving the expert's overflow
@@ -83,14 +86,16 @@ struct Smem {
     int* segs;    // [R] start of the rank's segment in the stream
     int* sege;    // [R] end of the rank's segment
     int* nsl;     // [R] slots the rank needs
-    int* fe;      // [R] first expert of the rank's segment (-1: none)
+    int* fe;      // [R] stream position of the rank's first item (-1: none)
     int* rload;   // [R] home rows before balancing
+    int* recv_at; // [R] the rank at each position of the receiving order
+    int* sege_at; // [R] segment end at each position of the receiving order
     int* scratch; // [2*SCAN_N*32 + 8]
     int* stash;   // [chunk] the block's picks (when stashed)
 };
 
 __host__ __device__ inline size_t smem_ints(int E, int R) {
-    return (size_t)NW * E + 8 * (size_t)E + 4 * ((size_t)E + 1) + 7 * (size_t)R +
+    return (size_t)NW * E + 11 * (size_t)E + 4 * ((size_t)E + 1) + 9 * (size_t)R +
            2 * SCAN_N * 32 + 8;
 }
 
@@ -105,8 +110,11 @@ __device__ inline Smem carve(int* base, int E, int R) {
     s.nzlist = p; p += E;
     s.pc = p; p += E + 1;
     s.pk = p; p += E + 1;
-    s.os = p; p += E + 1;
-    s.nzr = p; p += E + 1;
+    s.ov = p; p += E;
+    s.item_at = p; p += E;
+    s.osi = p; p += E + 1;
+    s.nzri = p; p += E + 1;
+    s.ose = p; p += E;
     s.kbase = p; p += E;
     s.rlo = p; p += E;
     s.rhi = p; p += E;
@@ -117,6 +125,8 @@ __device__ inline Smem carve(int* base, int E, int R) {
     s.nsl = p; p += R;
     s.fe = p; p += R;
     s.rload = p; p += R;
+    s.recv_at = p; p += R;
+    s.sege_at = p; p += R;
     s.scratch = p; p += 2 * SCAN_N * 32 + 8;
     s.stash = p;
     return s;
@@ -210,7 +220,7 @@ __device__ int balance(const PlanParams& p, Smem& s, int* misc) {
         if (ve) s.pc[e] = ex1[0];
         __syncthreads();
         if (ve) q = ex1[0] - s.pc[first];
-    } else if (ve) {
+    } else if (ve) {  // rules 1 and 2: lightest experts first
         for (int i = 0; i < Er; ++i) {
             const int e2 = first + i, c2 = s.cnt[e2];
             if (c2 < c || (c2 == c && e2 < e)) q += c2;
@@ -219,49 +229,106 @@ __device__ int balance(const PlanParams& p, Smem& s, int* misc) {
     const long long room = (long long)C - q;
     const int k = ve ? (int)min((long long)c, max(room, 0LL)) : 0;
     const int o = c - k;
-    const int flag = (ve && o > 0) ? 1 : 0;
-    int v[SCAN_N] = {c, k, o, flag}, ex[SCAN_N], tot[SCAN_N];
-    block_scan<SCAN_N>(v, ex, tot, s.scratch);
     if (ve) {
         s.kk[e] = k;
+        s.ov[e] = o;
+    }
+    // the overflow stream's expert order: index order (rules 0 and 1), or by
+    // decreasing overflow, ties to the lower index (rule 2)
+    int ip = e;
+    if (p.rule == MOONEP_RULE_LARGEST_FIRST) {
+        __syncthreads();
+        if (ve) {
+            ip = 0;
+            for (int e2 = 0; e2 < E; ++e2) {
+                const int o2 = s.ov[e2];
+                ip += (o2 > o) || (o2 == o && e2 < e);
+            }
+        }
+    }
+    if (ve) s.item_at[ip] = e;
+    __syncthreads();
+    // scans: c and k over experts (index order), o and "has overflow" over
+    // the stream positions
+    const int ei = ve ? s.item_at[tid] : 0;
+    const int oi = ve ? s.ov[ei] : 0;
+    const int fi = (ve && oi > 0) ? 1 : 0;
+    int v[SCAN_N] = {c, k, oi, fi}, ex[SCAN_N], tot[SCAN_N];
+    block_scan<SCAN_N>(v, ex, tot, s.scratch);
+    if (ve) {
         s.pc[e] = ex[0];
         s.pk[e] = ex[1];
-        s.os[e] = ex[2];
-        s.nzr[e] = ex[3];
-        if (flag) s.nzlist[ex[3]] = e;
+        s.osi[tid] = ex[2];
+        s.nzri[tid] = ex[3];
+        s.ose[ei] = ex[2];
+        if (fi) s.nzlist[ex[3]] = ei;
     }
     if (tid == 0) {
         s.pc[E] = tot[0];
         s.pk[E] = tot[1];
-        s.os[E] = tot[2];
-        s.nzr[E] = tot[3];
+        s.osi[E] = tot[2];
+        s.nzri[E] = tot[3];
     }
     __syncthreads();
 
-    // ranks: kept rows, deficits, segments, slots -- one warp, 32 ranks a step
+    // ranks, one warp, 32 ranks a step: kept rows and deficits; the receiving
+    // order (rank order, or by decreasing deficit, ties to the lower index,
+    // for rule 2); segments in that order; slots per rank
     if (warp == 0) {
-        int carry = 0, fail_r = -1, fail_n = 0;
         for (int r0 = 0; r0 < R; r0 += 32) {
             const int r = r0 + lane;
-            const bool vr = r < R;
-            const int kept = vr ? s.pk[(r + 1) * Er] - s.pk[r * Er] : 0;
-            const int load = vr ? s.pc[(r + 1) * Er] - s.pc[r * Er] : 0;
-            const int d = vr ? C - kept : 0;
+            if (r < R) {
+                const int kept = s.pk[(r + 1) * Er] - s.pk[r * Er];
+                s.kept[r] = kept;
+                s.rload[r] = s.pc[(r + 1) * Er] - s.pc[r * Er];
+                s.def[r] = C - kept;
+            }
+        }
+        __syncwarp();
+        for (int r0 = 0; r0 < R; r0 += 32) {
+            const int r = r0 + lane;
+            if (r < R) {
+                int rp = r;
+                if (p.rule == MOONEP_RULE_LARGEST_FIRST) {
+                    const int d = s.def[r];
+                    rp = 0;
+                    for (int r2 = 0; r2 < R; ++r2) {
+                        const int d2 = s.def[r2];
+                        rp += (d2 > d) || (d2 == d && r2 < r);
+                    }
+                }
+                s.recv_at[rp] = r;
+            }
+        }
+        __syncwarp();
+        int carry = 0;
+        for (int i0 = 0; i0 < R; i0 += 32) {
+            const int i = i0 + lane;
+            const int r = i < R ? s.recv_at[i] : 0;
+            const int d = i < R ? s.def[r] : 0;
             const int incl = warp_incl_scan(d, lane);
             const int segs = carry + incl - d;
             carry += __shfl_sync(0xffffffffu, incl, 31);
-            int nsl = 0, fe = -1;
-            if (vr && d > 0) {
-                fe = upper_bound(s.os, E, segs) - 1;
-                const int le = upper_bound(s.os, E, segs + d - 1) - 1;
-                nsl = s.nzr[le] - s.nzr[fe] + 1;
-            }
-            if (vr) {
-                s.kept[r] = kept;
-                s.rload[r] = load;
-                s.def[r] = d;
+            if (i < R) {
                 s.segs[r] = segs;
                 s.sege[r] = segs + d;
+                s.sege_at[i] = segs + d;
+            }
+        }
+        __syncwarp();
+        int fail_r = -1, fail_n = 0;
+        for (int r0 = 0; r0 < R; r0 += 32) {
+            const int r = r0 + lane;
+            const bool vr = r < R;
+            int nsl = 0, fe = -1;
+            const int d = vr ? s.def[r] : 0;
+            if (vr && d > 0) {
+                const int segs = s.segs[r];
+                fe = upper_bound(s.osi, E, segs) - 1;
+                const int le = upper_bound(s.osi, E, segs + d - 1) - 1;
+                nsl = s.nzri[le] - s.nzri[fe] + 1;
+            }
+            if (vr) {
                 s.nsl[r] = nsl;
                 s.fe[r] = fe;
             }
@@ -285,15 +352,16 @@ __device__ int balance(const PlanParams& p, Smem& s, int* misc) {
 __device__ __forceinline__ int place(const PlanParams& p, const Smem& s, int e, int pos) {
     const int k = s.kk[e];
     if (pos < k) return s.kbase[e] + pos;
-    const int sidx = s.os[e] + pos - k;
-    int lo = s.rlo[e], hi = s.rhi[e] + 1;  // the receiving rank lies in [rlo, rhi]
+    const int sidx = s.ose[e] + pos - k;
+    // the receiving position lies in [rlo, rhi] of the receiving order
+    int lo = s.rlo[e], hi = s.rhi[e] + 1;
     while (lo < hi) {
         const int mid = (lo + hi) >> 1;
-        if (s.sege[mid] <= sidx) lo = mid + 1;
+        if (s.sege_at[mid] <= sidx) lo = mid + 1;
         else hi = mid;
     }
-    const int rho = lo;
-    if (rho >= p.R) return -1;
+    if (lo >= p.R) return -1;
+    const int rho = s.recv_at[lo];
     return rho * p.C + s.kept[rho] + (sidx - s.segs[rho]);
 }
 
@@ -437,7 +505,7 @@ __global__ void __launch_bounds__(THREADS, 1) plan_kernel(PlanParams p) {
     for (int r = b; r < R; r += G) {
         const int kept = s.kept[r], d = s.def[r], segs = s.segs[r], sege = s.sege[r];
         const int nsl = s.nsl[r], fe = s.fe[r];
-        const int nz0 = fe >= 0 ? s.nzr[fe] : 0;
+        const int nz0 = fe >= 0 ? s.nzri[fe] : 0;
         const int rbase = s.pk[r * Er];
         for (int g = tid; g < E + B; g += THREADS) {
             int v;
@@ -448,7 +516,7 @@ __global__ void __launch_bounds__(THREADS, 1) plan_kernel(PlanParams p) {
                 const int j = g - E;
                 if (j < nsl) {
                     const int e = s.nzlist[nz0 + j];
-                    const int end = min(s.os[e] + (s.cnt[e] - s.kk[e]), sege);
+                    const int end = min(s.ose[e] + s.ov[e], sege);
                     v = kept + end - segs;
                 } else {
                     v = kept + d;
@@ -471,9 +539,9 @@ __global__ void __launch_bounds__(THREADS, 1) plan_kernel(PlanParams p) {
         }
         const int first = (e / Er) * Er;
         s.kbase[e] = (e / Er) * p.C + (s.pk[e] - s.pk[first]);
-        const int o = s.cnt[e] - s.kk[e];
-        s.rlo[e] = o > 0 ? upper_bound(s.sege, R, s.os[e]) : 0;
-        s.rhi[e] = o > 0 ? upper_bound(s.sege, R, s.os[e] + o - 1) : 0;
+        const int o = s.ov[e];
+        s.rlo[e] = o > 0 ? upper_bound(s.sege_at, R, s.ose[e]) : 0;
+        s.rhi[e] = o > 0 ? upper_bound(s.sege_at, R, s.ose[e] + o - 1) : 0;
     }
     __syncthreads();
 

@@ -25,6 +25,7 @@ PAYLOAD_BF16 = 0
 PAYLOAD_FP8 = 1
 RULE_INDEX_ORDER = 0
 RULE_KEEP_LIGHTEST = 1
+RULE_LARGEST_FIRST = 2
 EXPERT_IDENTITY = 0
 EXPERT_SCALE = 1
 MAX_E = 1024

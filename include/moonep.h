@@ -68,6 +68,8 @@ extern "C" {
 
 #define MOONEP_RULE_INDEX_ORDER 0   /* keep home rows in expert index order */
 #define MOONEP_RULE_KEEP_LIGHTEST 1 /* keep the lightest home experts whole */
+#define MOONEP_RULE_LARGEST_FIRST 2 /* keep as rule 1; hand the largest overflows to the
+                                       ranks with the largest deficits first */
 
 #define MOONEP_EXPERT_IDENTITY 0 /* stand-in expert: out = payload (fp8: dequantised) */
 #define MOONEP_EXPERT_SCALE 1    /* stand-in expert: out = bf16(v * (1 + e/E)) */
@@ -87,7 +89,7 @@ typedef struct moonep_config {
     int32_t H;             /* hidden size; a multiple of 8 (of 128 for fp8) */
     int32_t Hp;            /* expert intermediate size H' (weights only; 0 if unused) */
     int32_t payload;       /* MOONEP_PAYLOAD_* */
-    int32_t rule;          /* MOONEP_RULE_* */
+    int32_t rule;          /* MOONEP_RULE_* (0, 1 or 2) */
 } moonep_config;
 
 /* Byte sizes of every buffer a layer needs: the "buffer and prefetch-pool
@@ -164,15 +166,18 @@ int moonep_sizes(const moonep_config* cfg, moonep_sizes_t* out);
  * topk_idx: int32 [T, K] router picks, row-major, token-major (device).
  * Computes expert_count, rank_load, max count and maxvio; then, rule by rule:
  * each rank keeps its home rows (experts in index order, rows in (t, k)
- * order) up to C -- rule MOONEP_RULE_KEEP_LIGHTEST keeps lightest experts
- * whole instead -- the rows not kept form one stream in (rank, expert, t, k)
- * order that fills the under-full ranks in rank order to exactly C rows each;
+ * order) up to C -- rules MOONEP_RULE_KEEP_LIGHTEST and _LARGEST_FIRST keep
+ * the lightest experts whole instead -- the rows not kept form one stream,
+ * expert by expert (index order; for _LARGEST_FIRST by decreasing overflow,
+ * ties to the lower index), each expert's rows in (t, k) order, that fills
+ * the under-full ranks (in rank order; for _LARGEST_FIRST by decreasing
+ * deficit, ties to the lower rank) to exactly C rows each;
  * every distinct expert a rank receives takes one slot, in order of first
  * appearance; the kept rows come first in a rank's buffer, in expert order,
  * then the slot groups in slot order.  cu_seqlens[r][g] is the end row of
  * group g (experts 0..E-1, then slots E..E+B-1) in rank r's buffer; its last
  * entry is C.
- * A rank needing more than B slots sets status SLOT_BUDGET with the first
+ * A rank needing more than B slots sets status SLOT_BUDGET with the lowest
  * failing rank and its slot count; an index outside [0, E) sets BAD_INDEX.
  * Then only expert_count, rank_load, max count and maxvio are defined.
  * One memset of the status block plus one kernel; no host synchronisation. */

@@ -173,15 +173,19 @@ void oracle_e4m3_from_f32_array(const float* in, uint8_t* out, int64_t n)
  *      fit when the experts are filled lightest first (ascending
  *      (cnt, index)); the kept rows of an expert are its first ones in
  *      (t, k) order, and the kept rows are laid out in expert index order.
- *  O3  the overflow stream is every rank's rows that were not kept, rank
- *      by rank, expert by expert, in (t, k) order.
- *  O4  walking the ranks in order, each rank with a deficit C - kept[r]
- *      takes the next deficit rows of the stream, placed after its kept
- *      rows in stream order.
+ *  O3  the overflow stream is every rank's rows that were not kept, expert
+ *      by expert (rank by rank for rules 0 and 1, i.e. expert index order;
+ *      by decreasing overflow count, ties to the lower index, for rule 2),
+ *      each expert's rows in (t, k) order.
+ *  O4  walking the ranks in order (rules 0 and 1: index order; rule 2:
+ *      decreasing deficit, ties to the lower index), each rank with a
+ *      deficit C - kept[r] takes the next deficit rows of the stream, placed
+ *      after its kept rows in stream order.  Rule 2 keeps rows as rule 1
+ *      does.
  *  O5  on a receiving rank, each distinct expert of its segment takes one
  *      slot, in order of first appearance.  A rank that needs more than B
  *      slots fails the plan (status ORACLE_SLOT_BUDGET; *fail_rank is the
- *      first such rank, *fail_slots the slots it needs); then only O1's
+ *      lowest such rank, *fail_slots the slots it needs); then only O1's
  *      outputs and rank_load are defined.
  *  O6  cu_seqlens[r][g] is the inclusive prefix sum of the row counts of
  *      groups g = 0..E+B-1: group g < E holds rank r's kept rows of expert
@@ -203,7 +207,7 @@ int oracle_plan(int R, int S, int E, int K, int B, int rule,
                 int32_t* fail_rank, int32_t* fail_slots)
 {
     if (R <= 0 || S <= 0 || E <= 0 || K <= 0 || B < 0 || E % R != 0 ||
-        (rule != 0 && rule != 1))
+        rule < 0 || rule > 2)
         return ORACLE_INVALID;
     const int64_t T = (int64_t)R * S, P = T * K, C = (int64_t)S * K;
     const int Er = E / R;
@@ -245,10 +249,14 @@ int oracle_plan(int R, int S, int E, int K, int B, int rule,
     int32_t* stream_e = (int32_t*)malloc(sizeof(int32_t) * (size_t)P);
     int32_t* row_group = (int32_t*)malloc(sizeof(int32_t) * (size_t)P);
     int64_t* gcount = (int64_t*)malloc(sizeof(int64_t) * (size_t)(E + B));
+    int* xorder = (int*)malloc(sizeof(int) * (size_t)E);
+    int* rorder = (int*)malloc(sizeof(int) * (size_t)R);
+    int* rslots = (int*)malloc(sizeof(int) * (size_t)R);
     if (!first || !fillpos || !rows_of || !kept_n || !order || !next_row ||
-        !stream || !stream_e || !row_group || !gcount) {
+        !stream || !stream_e || !row_group || !gcount || !xorder || !rorder || !rslots) {
         free(first); free(fillpos); free(rows_of); free(kept_n); free(order);
         free(next_row); free(stream); free(stream_e); free(row_group); free(gcount);
+        free(xorder); free(rorder); free(rslots);
         return ORACLE_INVALID;
     }
     first[0] = 0;
@@ -263,7 +271,7 @@ int oracle_plan(int R, int S, int E, int K, int B, int rule,
     for (int r = 0; r < R; ++r) {
         for (int i = 0; i < Er; ++i)
             order[i] = r * Er + i; /* rule 0: index order */
-        if (rule == 1) {
+        if (rule >= 1) {
             /* lightest first: insertion sort by (cnt, index) */
             for (int i = 1; i < Er; ++i) {
                 int cur = order[i], j = i - 1;
@@ -299,57 +307,101 @@ int oracle_plan(int R, int S, int E, int K, int B, int rule,
         }
     }
 
-    /* O3: the overflow stream. */
-    int64_t nstream = 0;
-    for (int r = 0; r < R; ++r)
-        for (int e = r * Er; e < (r + 1) * Er; ++e)
-            for (int64_t i = kept_n[e]; i < expert_count[e]; ++i) {
-                stream[nstream] = rows_of[first[e] + i];
-                stream_e[nstream] = e;
-                ++nstream;
+    /* O3: the overflow stream: each expert's rows that were not kept, in
+     * (t, k) order.  Rules 0 and 1 take the experts in index order (which is
+     * rank order, since ranks own contiguous experts); rule 2 takes them in
+     * order of decreasing overflow count, ties to the lower index. */
+    for (int e = 0; e < E; ++e)
+        xorder[e] = e;
+    if (rule == 2) {
+        for (int i = 1; i < E; ++i) {
+            int cur = xorder[i], j = i - 1;
+            int64_t oc = expert_count[cur] - kept_n[cur];
+            while (j >= 0 && (expert_count[xorder[j]] - kept_n[xorder[j]] < oc ||
+                              (expert_count[xorder[j]] - kept_n[xorder[j]] == oc && xorder[j] > cur))) {
+                xorder[j + 1] = xorder[j];
+                --j;
             }
+            xorder[j + 1] = cur;
+        }
+    }
+    int64_t nstream = 0;
+    for (int i = 0; i < E; ++i) {
+        int e = xorder[i];
+        for (int64_t k = kept_n[e]; k < expert_count[e]; ++k) {
+            stream[nstream] = rows_of[first[e] + k];
+            stream_e[nstream] = e;
+            ++nstream;
+        }
+    }
 
-    /* O4 + O5: cut the stream, assign slots, place the segment rows. */
-    int status = ORACLE_OK;
+    /* O4: the receiving order.  Rules 0 and 1 walk the ranks in index
+     * order; rule 2 in order of decreasing deficit C - kept, ties to the
+     * lower index.  Ranks without a deficit take nothing. */
+    for (int r = 0; r < R; ++r)
+        rorder[r] = r;
+    if (rule == 2) {
+        for (int i = 1; i < R; ++i) {
+            int cur = rorder[i], j = i - 1;
+            int64_t dc = C - next_row[cur];
+            while (j >= 0 && (C - next_row[rorder[j]] < dc ||
+                              (C - next_row[rorder[j]] == dc && rorder[j] > cur))) {
+                rorder[j + 1] = rorder[j];
+                --j;
+            }
+            rorder[j + 1] = cur;
+        }
+    }
+
+    /* O4 + O5: cut the stream in the receiving order, assign slots, place
+     * the segment rows. */
+    for (int64_t i = 0; i < (int64_t)R * B; ++i)
+        slot_expert[i] = -1;
     int64_t pos = 0;
-    for (int r = 0; r < R && status == ORACLE_OK; ++r) {
-        for (int j = 0; j < B; ++j)
-            slot_expert[(int64_t)r * B + j] = -1;
+    for (int i = 0; i < R; ++i) {
+        int r = rorder[i];
         int64_t deficit = C - next_row[r];
         int nslots = 0;
         int last_e = -1;
-        /* first pass: count distinct experts (the stream is expert-sorted,
-         * so a new expert shows up as a change of expert id) */
-        for (int64_t i = 0; i < deficit; ++i) {
-            int e = stream_e[pos + i];
+        /* the stream is grouped by expert, so a new expert shows up as a
+         * change of expert id */
+        for (int64_t q = 0; q < deficit; ++q) {
+            int e = stream_e[pos + q];
             if (e != last_e) {
                 ++nslots;
                 last_e = e;
             }
         }
-        if (nslots > B) {
-            status = ORACLE_SLOT_BUDGET;
-            *fail_rank = r;
-            *fail_slots = nslots;
-            break;
-        }
-        int j = -1;
-        last_e = -1;
-        for (int64_t i = 0; i < deficit; ++i) {
-            int e = stream_e[pos + i];
-            if (e != last_e) {
-                ++j;
-                slot_expert[(int64_t)r * B + j] = e;
-                last_e = e;
+        rslots[r] = nslots;
+        if (nslots <= B) {
+            int j = -1;
+            last_e = -1;
+            for (int64_t q = 0; q < deficit; ++q) {
+                int e = stream_e[pos + q];
+                if (e != last_e) {
+                    ++j;
+                    slot_expert[(int64_t)r * B + j] = e;
+                    last_e = e;
+                }
+                int32_t p = stream[pos + q];
+                int64_t row = next_row[r]++;
+                dst_row[p] = (int32_t)(r * C + row);
+                src_of_row[r * C + row] = p;
+                row_group[r * C + row] = E + j;
             }
-            int32_t p = stream[pos + i];
-            int64_t row = next_row[r]++;
-            dst_row[p] = (int32_t)(r * C + row);
-            src_of_row[r * C + row] = p;
-            row_group[r * C + row] = E + j;
         }
         pos += deficit;
     }
+    /* a rank that needs more than B slots fails the plan: report the lowest
+     * such rank and the slots it needs */
+    int status = ORACLE_OK;
+    for (int r = 0; r < R; ++r)
+        if (rslots[r] > B) {
+            status = ORACLE_SLOT_BUDGET;
+            *fail_rank = r;
+            *fail_slots = rslots[r];
+            break;
+        }
 
     /* O6: cu_seqlens from the rows actually placed. */
     if (status == ORACLE_OK) {
@@ -368,6 +420,7 @@ int oracle_plan(int R, int S, int E, int K, int B, int rule,
 
     free(first); free(fillpos); free(rows_of); free(kept_n); free(order);
     free(next_row); free(stream); free(stream_e); free(row_group); free(gcount);
+    free(xorder); free(rorder); free(rslots);
     return status;
 }
 

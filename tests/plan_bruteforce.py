@@ -11,6 +11,9 @@ through index arithmetic.  Both follow the same written rule:
   one stream in (rank, expert, token, k) order; ranks with room take the next
   rows of the stream in rank order; each distinct expert a rank receives
   takes one slot in order of first appearance; more than B slots fails.
+  Rule 2 keeps rows as rule 1, orders the stream's experts by decreasing
+  overflow count (ties: lower index) and walks the receiving ranks by
+  decreasing deficit (ties: lower index).
 """
 from collections import Counter
 
@@ -35,7 +38,7 @@ def brute_plan(idx, R, S, E, K, B, rule=0):
         home = sorted(tr for tr in triples if tr[0] // Er == r)
         if rule == 0:
             kept, over = home[:C], home[C:]
-        else:
+        else:  # rules 1 and 2: lightest experts kept first
             experts = sorted(range(r * Er, (r + 1) * Er), key=lambda e: (counts[e], e))
             room = C
             quota = {}
@@ -53,9 +56,16 @@ def brute_plan(idx, R, S, E, K, B, rule=0):
         rows[r] = [(tr[0], tr) for tr in kept]
         stream.extend(over)
 
+    if rule == 2:
+        over_n = Counter(tr[0] for tr in stream)
+        stream.sort(key=lambda tr: (-over_n[tr[0]], tr[0], tr[1], tr[2]))
+        walk = sorted(range(R), key=lambda r: (-(C - len(rows[r])), r))
+    else:
+        walk = list(range(R))
     slot_expert = [[-1] * B for _ in range(R)]
     at = 0
-    for r in range(R):
+    failing = []
+    for r in walk:
         need = C - len(rows[r])
         seg = stream[at:at + need]
         at += need
@@ -64,12 +74,16 @@ def brute_plan(idx, R, S, E, K, B, rule=0):
             if tr[0] not in distinct:
                 distinct.append(tr[0])
         if len(distinct) > B:
-            return dict(status=3, fail_rank=r, fail_slots=len(distinct), expert_count=counts,
-                        rank_load=rank_load, max_count=max_count, maxvio=maxvio)
+            failing.append((r, len(distinct)))
+            continue
         for j, e in enumerate(distinct):
             slot_expert[r][j] = e
         rows[r].extend((E + distinct.index(tr[0]), tr) for tr in seg)
     assert at == len(stream)
+    if failing:
+        r, n = min(failing)
+        return dict(status=3, fail_rank=r, fail_slots=n, expert_count=counts,
+                    rank_load=rank_load, max_count=max_count, maxvio=maxvio)
 
     cu = []
     dst_row = [[None] * K for _ in range(T)]

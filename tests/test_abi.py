@@ -64,7 +64,7 @@ def test_version_and_sizes(m):
     (dict(S=1 << 28, K=8, R=1), "2\\^31"),
     (dict(S=0), "positive"),
     (dict(B=-1), "non-negative"),
-    (dict(rule=2), "rule"),
+    (dict(rule=3), "rule"),
 ])
 def test_config_rejected(m, bad, msg):
     d = dict(R=2, S=8, E=4, K=2, B=2, H=64, Hp=0, payload=0, rule=0)

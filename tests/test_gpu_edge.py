@@ -43,14 +43,14 @@ def test_degenerate_and_ragged(shape):
     cfgd = _cfg(R, S, E, K, B, H)
     for seed in range(3):
         idx, w = wl.routing(cfgd, seed=seed)
-        for rule in (0, 1):
+        for rule in (0, 1, 2):
             _full_check(cfgd, idx, w, seed=seed, rule=rule)
 
 
 def test_largest_E_and_R():
     cfgd = _cfg(128, 16, 1024, 8, 16, 64, alpha=1.2)
     idx, w = wl.routing(cfgd, seed=0)
-    for rule in (0, 1):
+    for rule in (0, 1, 2):
         _full_check(cfgd, idx, w, rule=rule, expert="identity")
 
 

@@ -57,7 +57,7 @@ def _check_full_small(cfgd, idx, w, x_dev, rule, expert):
     return out, o
 
 
-@pytest.mark.parametrize("rule", [0, 1])
+@pytest.mark.parametrize("rule", [0, 1, 2])
 def test_random_small_configs(rule):
     rng = np.random.default_rng(7 + rule)
     statuses = set()
@@ -71,16 +71,16 @@ def test_random_small_configs(rule):
 
 
 @pytest.mark.parametrize("expert", ["identity", "scale"])
-def test_c1_full(expert):
+def test_tiny_full(expert):
     cfgd = wl.WORKLOADS["tiny"]
     for seed in range(3):
         idx, w = wl.routing(cfgd, seed=seed)
         x = wl.hidden(cfgd["R"] * cfgd["S"], cfgd["H"], seed=seed).cuda()
-        for rule in (0, 1):
+        for rule in (0, 1, 2):
             _check_full_small(cfgd, idx, w, x, rule, expert)
 
 
-def test_c2_full():
+def test_uniform_full():
     cfgd = wl.WORKLOADS["uniform"]
     idx, w = wl.routing(cfgd, seed=0)
     x = wl.hidden(cfgd["R"] * cfgd["S"], cfgd["H"], seed=0).cuda()
@@ -151,26 +151,27 @@ def _path_tokens_rows(cfgd, x_rows, w_rows, o, tokens, src_c, expert, payload):
 
 
 @pytest.mark.parametrize("alpha", [0.0, 0.5, 1.0, 1.5])
-@pytest.mark.parametrize("rule", [0, 1])
-def test_c3_zipf_sweep(alpha, rule):
+@pytest.mark.parametrize("rule", [0, 1, 2])
+def test_zipf_sweep(alpha, rule):
     cfgd = wl.WORKLOADS["zipf"]
     idx, w, x = routing_and_x(cfgd, seed=0, alpha=alpha)
     out, o = _check_large(cfgd, idx, w, x, rule, "scale")
-    if rule == 1:
+    if rule >= 1:
         assert o["status"] == 0  # keep-lightest fits the slot budget at every skew
 
 
-def test_c4_adversarial():
+@pytest.mark.parametrize("rule", [0, 2])
+def test_hot_adversarial(rule):
     cfgd = wl.WORKLOADS["hot"]
     idx, w, x = routing_and_x(cfgd, seed=0)
-    out, o = _check_large(cfgd, idx, w, x, 0, "identity", n_sample=256)
+    out, o = _check_large(cfgd, idx, w, x, rule, "identity", n_sample=256)
     assert o["status"] == 0
     assert o["maxvio"] > 100  # half of all picks on one expert
     del out
     torch.cuda.empty_cache()
 
 
-def test_c5_fp8():
+def test_fp8_workload():
     cfgd = wl.WORKLOADS["fp8"]
     idx, w, x = routing_and_x(cfgd, seed=0)
     out, o = _check_large(cfgd, idx, w, x, 0, "identity", n_sample=256)
@@ -220,5 +221,5 @@ def test_small_fp8_full(H):
         x = wl.hidden(cfgd["R"] * cfgd["S"], H, seed=it).cuda()
         if it == 0:
             x[0].zero_()  # a zero row: scale 1, zero codes
-        for rule in (0, 1):
+        for rule in (0, 1, 2):
             _check_full_small(cfgd, idx, w, x, rule, "scale" if it % 2 else "identity")

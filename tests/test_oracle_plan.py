@@ -57,7 +57,7 @@ def test_golden_plans(oracle_mod, case):
     assert ref["dst_row"] == case["dst_row"]
 
 
-@pytest.mark.parametrize("rule", [0, 1])
+@pytest.mark.parametrize("rule", [0, 1, 2])
 def test_exhaustive_distinct_R2_S2_E4_K2(oracle_mod, rule):
     """Every routing of 4 tokens over 4 experts with 2 distinct picks, with
     B = 1 (every plan fits: one over-full rank of two experts overflows at
@@ -86,12 +86,12 @@ def test_sampled_duplicates_R2_S3_E4_K2(oracle_mod):
     for it in range(3000):
         B = 1 + it % 2
         idx = rng.integers(0, E, (R * S, K)).astype(np.int32)
-        got = _cmp_with_brute(oracle_mod, idx, R, S, E, K, B, it % 3 == 0)
+        got = _cmp_with_brute(oracle_mod, idx, R, S, E, K, B, it % 3)
         if got["status"] == 0:
             check_plan_invariants(got, idx, R, S, E, K, B)
 
 
-@pytest.mark.parametrize("rule", [0, 1])
+@pytest.mark.parametrize("rule", [0, 1, 2])
 def test_random_small_configs(oracle_mod, rule):
     rng = np.random.default_rng(100 + rule)
     seen = set()
@@ -154,7 +154,7 @@ def test_maxvio_closed_forms(oracle_mod):
 
 @pytest.mark.parametrize("name,alpha", [("tiny", None), ("uniform", None), ("zipf", 0.0), ("zipf", 0.5),
                                         ("zipf", 1.0), ("zipf", 1.5)])
-@pytest.mark.parametrize("rule", [0, 1])
+@pytest.mark.parametrize("rule", [0, 1, 2])
 def test_workload_plans_invariants(oracle_mod, name, alpha, rule):
     cfg = wl.WORKLOADS[name]
     R, S, E, K, B = (cfg[k] for k in ("R", "S", "E", "K", "B"))
@@ -168,3 +168,23 @@ def test_workload_plans_invariants(oracle_mod, name, alpha, rule):
         check_plan_invariants(got, idx, R, S, E, K, B, rule)
     else:
         assert got["fail_slots"] > B
+
+
+def test_rule2_needs_fewer_slots_on_the_workloads(oracle_mod):
+    """Rule 2 (stream by decreasing overflow, ranks by decreasing deficit)
+    lowers the most slots any rank needs: measured on these seeded routings,
+    rule 1 -> rule 2 goes 5 -> 3 (zipf a=0.5), 5 -> 3 (fp8), 4 -> 2 (hot),
+    5 -> 3 (uniform)."""
+    import numpy as np
+    for name, alpha, seed, want in [("zipf", 0.5, 3, (5, 3)), ("fp8", None, 3, (5, 3)),
+                                    ("hot", None, 0, (4, 2)), ("uniform", None, 0, (5, 3))]:
+        cfg = wl.WORKLOADS[name]
+        R, S, E, K = cfg["R"], cfg["S"], cfg["E"], cfg["K"]
+        idx, _ = wl.routing(cfg, seed=seed, alpha=alpha)
+        need = []
+        for rule in (1, 2):
+            pl = oracle_mod.plan(R, S, E, K, 64, idx, rule=rule)
+            assert pl["status"] == 0
+            check_plan_invariants(pl, idx, R, S, E, K, 64, rule)
+            need.append(int((pl["slot_expert"] >= 0).sum(axis=1).max()))
+        assert tuple(need) == want, (name, need)
