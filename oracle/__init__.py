@@ -61,6 +61,10 @@ def lib():
         L.oracle_grad_reduce.argtypes = [ci, ci, ci, cl, i32p, f32p, f32p]
         L.oracle_combine_backward_tokens.argtypes = [ci, ci, cl, f32p, u16p, u16p, u16p, f64p]
         L.oracle_dispatch_backward_tokens.argtypes = [ci, ci, cl, u16p, u16p]
+        L.oracle_bf16_from_f64_array.argtypes = [f64p, u16p, cl]
+        L.oracle_row_group.argtypes = [ci, ci, i32p, cl]
+        L.oracle_row_group.restype = ci
+        L.oracle_expert_gemm_rows.argtypes = [ci, ci, cl, u16p, i32p, u16p, u16p, f64p, f64p]
         _lib = L
     return _lib
 
@@ -271,3 +275,40 @@ def dispatch_backward_tokens(d_recv_bits):
     dx = np.empty((n, H), np.uint16)
     lib().oracle_dispatch_backward_tokens(K, H, n, d_recv_bits.reshape(-1), dx.reshape(-1))
     return dx
+
+
+# ---------------------------------------------------------------- expert GEMM
+def bf16_from_f64(v):
+    """double -> bf16 bits, one round-to-nearest-even on the double."""
+    v = _c(v, np.float64)
+    out = np.empty(v.shape, np.uint16)
+    lib().oracle_bf16_from_f64_array(v.reshape(-1), out.reshape(-1), v.size)
+    return out
+
+
+def row_groups(E, B, C, cu_seqlens, rows):
+    """(rank, group) of each global row index rank*C + i under a plan."""
+    cu = _c(cu_seqlens, np.int32).reshape(-1, E + B)
+    rows = np.asarray(rows, np.int64)
+    ranks = rows // C
+    groups = np.empty(rows.shape, np.int64)
+    for n, (r, i) in enumerate(zip(ranks.tolist(), (rows % C).tolist())):
+        groups[n] = lib().oracle_row_group(E, B, np.ascontiguousarray(cu[r]), i)
+    return ranks, groups
+
+
+def expert_gemm_rows(x_bits, mat, w_bits):
+    """x [n,H] bf16 bits, mat [n] index into w [nmat,H,Hp] bf16 bits ->
+    (y [n,Hp] bf16 bits, s [n,Hp] float64 sums, sabs [n,Hp] sum |x w|)."""
+    x_bits = _c(x_bits, np.uint16)
+    mat = _c(mat, np.int32)
+    w_bits = _c(w_bits, np.uint16)
+    n, H = x_bits.shape
+    _, H2, Hp = w_bits.shape
+    assert H2 == H and mat.shape == (n,)
+    y = np.empty((n, Hp), np.uint16)
+    s = np.empty((n, Hp), np.float64)
+    sabs = np.empty((n, Hp), np.float64)
+    lib().oracle_expert_gemm_rows(H, Hp, n, x_bits.reshape(-1), mat, w_bits.reshape(-1),
+                                  y.reshape(-1), s.reshape(-1), sabs.reshape(-1))
+    return y, s, sabs

@@ -649,3 +649,95 @@ void oracle_dispatch_backward_tokens(int K, int H, int64_t n, const uint16_t* d_
             dx[i * H + h] = oracle_bf16_from_f32(acc);
         }
 }
+
+/* ------------------------------------------------------------------ */
+/* Grouped expert GEMM (the consumer of a plan)                        */
+/* ------------------------------------------------------------------ */
+
+/* double -> bfloat16 with one rounding, to nearest, ties to even, taken on
+ * the double itself (no intermediate binary32).  bf16 keeps 8 significant
+ * bits for exponents down to -126 and a fixed spacing of 2^-133 below.  A
+ * magnitude a in [2^(e-1), 2^e) (frexp's e) lies on the grid of spacing
+ * 2^(max(e, -125) - 8); a / spacing is rounded to an integer, ties to even,
+ * and scaled back.  A result of 2^128 or more is infinity; NaN stays NaN. */
+uint16_t oracle_bf16_from_f64(double v)
+{
+    if (isnan(v))
+        return 0x7fc0;
+    uint16_t sign = signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    if (isinf(a))
+        return sign | 0x7f80;
+    if (a == 0.0)
+        return sign;
+    int e;
+    frexp(a, &e);
+    int q = (e > -125 ? e : -125) - 8;
+    double r = ldexp(round_half_even(ldexp(a, -q)), q);
+    if (r >= ldexp(1.0, 128))
+        return sign | 0x7f80;
+    float f = (float)r; /* exact: r has at most 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    return sign | (uint16_t)((u >> 16) & 0x7fffu);
+}
+
+void oracle_bf16_from_f64_array(const double* in, uint16_t* out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = oracle_bf16_from_f64(in[i]);
+}
+
+/* The group of rank r that holds row `row` of the rank: the g with
+ * cu_r[g-1] <= row < cu_r[g] (cu_seqlens are inclusive end offsets), or -1. */
+int oracle_row_group(int E, int B, const int32_t* cu_r, int64_t row)
+{
+    for (int g = 0; g < E + B; ++g)
+        if (row < cu_r[g])
+            return g;
+    return -1;
+}
+
+/* The framework's grouped GEMM over a plan ([ainovat], the framework-contract
+ * paragraph: it reads the contiguous [E+B, H, H'] weight tensor and picks
+ * each group's rows through cu_seqlens[E+B]).  A row of rank r in group g is
+ * multiplied by row g of rank r's weight view: g < E is home expert g, g >= E
+ * the replica in slot g - E.  For row i (the caller has resolved its matrix
+ * to mat[i] in w, [nmat][H][Hp]):
+ *   s[i][j] = sum_h x[i][h] * w[mat[i]][h][j]   in binary64, h ascending,
+ *   y[i][j] = bf16(s[i][j])                     one rounding, ties to even.
+ * A product of two bf16 values is exact in binary64, so s differs from the
+ * exact sum by binary64 rounding only (at most H * 2^-53 * sum_h |x w|).
+ * s and sabs (sum_h |x w|, for error bounds) are written when not NULL. */
+void oracle_expert_gemm_rows(int H, int Hp, int64_t n, const uint16_t* x, const int32_t* mat,
+                             const uint16_t* w, uint16_t* y, double* s, double* sabs)
+{
+    double* acc = (double*)malloc(sizeof(double) * (size_t)Hp * 2);
+    if (!acc)
+        return;
+    double* aab = acc + Hp;
+    for (int64_t i = 0; i < n; ++i) {
+        const uint16_t* wm = w + (int64_t)mat[i] * H * Hp;
+        for (int j = 0; j < Hp; ++j) {
+            acc[j] = 0.0;
+            aab[j] = 0.0;
+        }
+        for (int h = 0; h < H; ++h) {
+            double xv = (double)oracle_bf16_to_f32(x[i * H + h]);
+            const uint16_t* wr = wm + (int64_t)h * Hp;
+            for (int j = 0; j < Hp; ++j) {
+                double p = xv * (double)oracle_bf16_to_f32(wr[j]);
+                acc[j] += p;
+                aab[j] += fabs(p);
+            }
+        }
+        for (int j = 0; j < Hp; ++j) {
+            y[i * Hp + j] = oracle_bf16_from_f64(acc[j]);
+            if (s)
+                s[i * Hp + j] = acc[j];
+            if (sabs)
+                sabs[i * Hp + j] = aab[j];
+        }
+    }
+    free(acc);
+}
