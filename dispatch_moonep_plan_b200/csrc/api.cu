@@ -240,6 +240,31 @@ int moonep_expert_standin(const moonep_config* c, const moonep_plan_t* plan, con
     return MOONEP_OK;
 }
 
+int moonep_expert_gemm(const moonep_config* c, const moonep_plan_t* plan, const void* recv,
+                       const void* weights, void* out, moonep_stream_t stream) {
+    const char* fn = "moonep_expert_gemm";
+    if (const char* why = check_config(c)) return fail(MOONEP_ERR_INVALID_ARG, fn, why);
+    if (const char* why = check_plan(c, plan)) return fail(MOONEP_ERR_INVALID_ARG, fn, why);
+    if (c->payload != MOONEP_PAYLOAD_BF16)
+        return fail(MOONEP_ERR_INVALID_ARG, fn, "the expert GEMM takes the bf16 payload only");
+    if (c->H % 64 != 0) return fail(MOONEP_ERR_INVALID_ARG, fn, "H must be a multiple of 64");
+    if (c->Hp <= 0 || c->Hp % 128 != 0)
+        return fail(MOONEP_ERR_INVALID_ARG, fn, "Hp must be a positive multiple of 128");
+    if ((long long)c->R * (c->E + c->B) * c->H >= (1LL << 31))
+        return fail(MOONEP_ERR_INVALID_ARG, fn, "R*(E+B)*H must be below 2^31");
+    if (!recv || !weights || !out)
+        return fail(MOONEP_ERR_INVALID_ARG, fn, "recv, weights or out is NULL");
+    if (!aligned16(recv) || !aligned16(weights) || !aligned16(out))
+        return fail(MOONEP_ERR_INVALID_ARG, fn, "recv, weights and out must be 16-byte aligned");
+    if (!moonep::expert_gemm_fits(*c))
+        return fail(MOONEP_ERR_INVALID_ARG, fn, "too many (rank, group) pairs for shared memory");
+    const char* why = nullptr;
+    cudaError_t e = moonep::launch_expert_gemm(*c, *plan, recv, weights, out,
+                                               static_cast<cudaStream_t>(stream), &why);
+    if (e != cudaSuccess) return cuda_fail(fn, e, why);
+    return MOONEP_OK;
+}
+
 int moonep_prefetch(const moonep_config* c, const moonep_plan_t* plan, void* const* rank_weights,
                     int32_t elem_bytes, moonep_stream_t stream) {
     const char* fn = "moonep_prefetch";

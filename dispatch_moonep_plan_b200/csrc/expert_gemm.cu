@@ -1,0 +1,525 @@
+// expert_gemm.cu -- the grouped expert GEMM that consumes a plan: for every
+// rank r and every group g of its [E+B] groups, the rows [cu[r][g-1],
+// cu[r][g]) of rank r's dispatched block are multiplied by row g of rank r's
+// [E+B, H, H'] weight view.
+//
+// This is the consumer the pages put after dispatch: the framework's grouped
+// GEMM reads the contiguous [E+B, H, H'] weight tensor and selects the active
+// rows through cu_seqlens[E+B] ("Moonshot AI Open-Sources MoonEP ..." on
+// ainovat.com, the framework-contract paragraph; "MoonEP" on moses-y.github.io,
+// "What This Does").  The pages give no kernel for it; this one is written
+// for sm_100a:
+//
+//  - one persistent CTA per SM, 192 threads: warp 0 issues TMA loads, one
+//    thread of warp 1 issues tcgen05.mma, warps 2-5 drain the accumulator;
+//  - tile 128 rows x BN columns (BN = 256 when H' allows, else 128), k-block
+//    64: A = 128 x 64 bf16 rows of the dispatched block (K-major), B = 64 x BN
+//    of the weight row (H' contiguous, MN-major), both 128-byte swizzled;
+//  - the fp32 accumulator lives in tensor memory, two buffers of BN columns,
+//    so the epilogue of one tile overlaps the main loop of the next;
+//  - the epilogue reads 32 lanes x 32 columns per tcgen05.ld, rounds once to
+//    bf16 (round-to-nearest-even) and stores only the rows of the group.
+//
+// The tile list is built in each CTA from the plan: only the groups a plan
+// can fill are visited (rank r's E/R home experts and its B slots; every
+// other group of rank r is empty by construction of the plan), their m-tile
+// counts are scanned in shared memory and a tile index is mapped back to
+// (rank, group, m-tile, n-tile) by binary search.  Tiles go to CTAs
+// round-robin in (m-tile, n-tile) order, so the CTAs running at one time read
+// the same A rows and the same expert's weights from L2.
+//
+// Every wait is bounded by the library's wait limit (globaltimer).  A wait
+// that runs out raises a CTA-wide abort flag; each role then stops, the TMA
+// warp waits (bounded) for the loads it still has in flight, the MMA thread
+// waits (bounded) for its issued MMAs to finish, TMEM is released, and the
+// plan's status becomes MOONEP_STATUS_TIMEOUT.
+#include <cuda.h>
+
+#include <mutex>
+
+#include "internal.cuh"
+
+namespace moonep {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int THREADS = 192;
+constexpr int A_BYTES = BM * BK * 2;  // 16 KiB
+// dynamic shared memory a CTA may ask for: the 227 KiB opt-in limit less
+// room for the kernel's static shared variables
+constexpr int SMEM_LIMIT = 227 * 1024 - 256;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* b, int count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_test(uint64_t* b, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; "
+        "selp.u32 %0, 1, 0, p; }"
+        : "=r"(done)
+        : "r"(smem_u32(b)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Wait for the phase of `parity` to complete.  Gives up (returns false) when
+// another role has raised the abort flag or after `limit` ns, raising it.
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, unsigned long long limit,
+                                          volatile int* abort) {
+    const unsigned long long t0 = globaltimer_ns();
+    for (int it = 1;; ++it) {
+        if (mbar_test(b, parity)) return true;
+        if ((it & 63) == 0) {
+            if (*abort) return false;
+            if (globaltimer_ns() - t0 > limit) {
+                *abort = 1;
+                return false;
+            }
+        }
+    }
+}
+
+// The same wait without the abort check: used to drain in-flight work.
+__device__ __forceinline__ bool mbar_drain(uint64_t* b, uint32_t parity, unsigned long long limit) {
+    const unsigned long long t0 = globaltimer_ns();
+    for (int it = 1;; ++it) {
+        if (mbar_test(b, parity)) return true;
+        if ((it & 63) == 0 && globaltimer_ns() - t0 > limit) return false;
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor for tcgen05.mma: start, leading and stride
+// byte offsets (>> 4), descriptor version 1 (bits 46-47) and the 128-byte
+// swizzle mode (2 in bits 61-63).
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = (uint64_t)((addr >> 4) & 0x3fff);
+    d |= (uint64_t)((lbo >> 4) & 0x3fff) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3fff) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+// Arrive on `bar` once every tcgen05 operation this thread issued is done.
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    unsigned short a, b;
+    asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(a) : "f"(lo));
+    asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(b) : "f"(hi));
+    return (uint32_t)a | ((uint32_t)b << 16);
+}
+
+struct GemmArgs {
+    int R, C, E, B, Er, H, Hp;
+    const int32_t* cu;  // [R][E+B] inclusive row ends
+    int32_t* status;
+    uint16_t* y;  // [R*C, Hp] bf16
+    unsigned long long wait_ns;
+    int debug_stall;  // epilogue waits on a barrier nothing completes
+};
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(THREADS, 1)
+    expert_gemm_kernel(const __grid_constant__ CUtensorMap tmX,
+                       const __grid_constant__ CUtensorMap tmW, GemmArgs p) {
+    constexpr int B_BYTES = BK * BN * 2;
+    constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    constexpr int TMEM_COLS = 2 * BN;
+    // k-block of A: 128 rows x 128 B; one k-step (16 elements) = 32 B along a row.
+    // k-block of B: BN/64 column chunks of 64 k-rows x 128 B (8 KiB each); one
+    // k-step = 16 k-rows = 2 KiB; the next 64-column chunk is 8 KiB further.
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint64_t* full = (uint64_t*)(smem + STAGES * STAGE_BYTES);
+    uint64_t* empty = full + STAGES;
+    uint64_t* tfull = empty + STAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* drain = tempty + 2;
+    uint64_t* never = drain + 1;
+    uint32_t* tmem_slot = (uint32_t*)(never + 1);
+    int* wsum = (int*)(tmem_slot + 2);  // [THREADS / 32]
+    int* pre = wsum + 8;                // [npairs + 1] m-tile prefix
+    __shared__ volatile int abort_flag;
+    __shared__ int plan_status;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // one read per CTA: another CTA of this launch may raise TIMEOUT meanwhile
+    if (tid == 0) plan_status = load_status(p.status);
+    __syncthreads();
+    if (plan_status != MOONEP_STATUS_OK) return;
+
+    const int G = p.E + p.B;      // groups per rank
+    const int per = p.Er + p.B;   // groups a plan can fill per rank
+    const int npairs = p.R * per;
+    const int ntn = p.Hp / BN;
+    const int kblocks = p.H / BK;
+
+    if (tid == 0) {
+        abort_flag = 0;
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 4);
+        }
+        mbar_init(drain, 1);
+        mbar_init(never, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    // (rank, group) of pair i: home groups of the rank first, then its slots
+    auto pair_rg = [&](int i, int& r, int& g) {
+        r = i / per;
+        const int j = i - r * per;
+        g = j < p.Er ? r * p.Er + j : p.E + (j - p.Er);
+    };
+    // m-tile count of every pair, then an exclusive scan over the block
+    const int chunk = (npairs + THREADS - 1) / THREADS;
+    const int lo_i = min(npairs, tid * chunk), hi_i = min(npairs, lo_i + chunk);
+    int sum = 0;
+    for (int i = lo_i; i < hi_i; ++i) {
+        int r, g;
+        pair_rg(i, r, g);
+        const int hi = __ldg(p.cu + r * G + g);
+        const int lo = g ? __ldg(p.cu + r * G + g - 1) : 0;
+        const int c = (hi - lo + BM - 1) / BM;
+        pre[i] = c;
+        sum += c;
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    if (warp == 1) {  // TMEM: both accumulators (one warp allocates)
+        asm volatile(
+            "tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                smem_u32(tmem_slot)),
+            "r"(TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    __syncthreads();
+    int run = incl - sum;
+    for (int w = 0; w < warp; ++w) run += wsum[w];
+    for (int i = lo_i; i < hi_i; ++i) {
+        const int c = pre[i];
+        pre[i] = run;
+        run += c;
+    }
+    if (tid == THREADS - 1) pre[npairs] = run;
+    asm volatile("tcgen05.fence::before_thread_sync;");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;");
+    const uint32_t tmem = *tmem_slot;
+    const int total = pre[npairs] * ntn;
+
+    // tile -> pair, m-tile within the pair's group, n-tile
+    auto locate = [&](int tile, int& pair, int& mt, int& nt) {
+        const int mtile = tile / ntn;
+        nt = tile - mtile * ntn;
+        int lo = 0, hi = npairs;  // pre[lo] <= mtile < pre[hi]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (pre[mid] <= mtile)
+                lo = mid;
+            else
+                hi = mid;
+        }
+        pair = lo;
+        mt = mtile - pre[lo];
+    };
+
+    if (warp == 0) {
+        if (lane == 0) {  // TMA producer
+            int s = 0;
+            uint32_t ph = 0;
+            long long issued = 0;
+            for (int tile = blockIdx.x; tile < total && !abort_flag; tile += gridDim.x) {
+                int pair, mt, nt, r, g;
+                locate(tile, pair, mt, nt);
+                pair_rg(pair, r, g);
+                const int row0 = r * p.C + (g ? __ldg(p.cu + r * G + g - 1) : 0) + mt * BM;
+                const int wrow0 = (r * G + g) * p.H;
+                bool ok = true;
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(&empty[s], ph ^ 1, p.wait_ns, &abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_expect_tx(&full[s], STAGE_BYTES);
+                    uint8_t* a = smem + s * STAGE_BYTES;
+                    uint8_t* b = a + A_BYTES;
+                    tma_load_2d(a, &tmX, &full[s], kb * BK, row0);
+#pragma unroll
+                    for (int j = 0; j < BN / 64; ++j)
+                        tma_load_2d(b + j * 8192, &tmW, &full[s], nt * BN + 64 * j,
+                                    wrow0 + kb * BK);
+                    ++issued;
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1;
+                    }
+                }
+                if (!ok) break;
+            }
+            if (abort_flag) {
+                // load n went to stage n % STAGES in phase (n / STAGES) & 1;
+                // wait for the last STAGES of them to land before leaving
+                for (long long n = issued > STAGES ? issued - STAGES : 0; n < issued; ++n)
+                    mbar_drain(&full[n % STAGES], (uint32_t)((n / STAGES) & 1), p.wait_ns);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {  // MMA issuer
+            // kind::f16 instruction descriptor: D f32 (bit 4), A bf16 (bit 7),
+            // B bf16 (bit 10), A K-major (bit 15 = 0), B MN-major (bit 16),
+            // N >> 3 at bit 17, M >> 4 at bit 24
+            const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
+                                   ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+            int s = 0;
+            uint32_t ph = 0;
+            int acc = 0;
+            uint32_t acc_ph = 0;
+            bool any = false;
+            for (int tile = blockIdx.x; tile < total && !abort_flag; tile += gridDim.x) {
+                if (!mbar_wait(&tempty[acc], acc_ph ^ 1, p.wait_ns, &abort_flag)) break;
+                asm volatile("tcgen05.fence::after_thread_sync;");
+                const uint32_t d = tmem + acc * BN;
+                bool ok = true;
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(&full[s], ph, p.wait_ns, &abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    asm volatile("tcgen05.fence::after_thread_sync;");
+                    const uint32_t a = smem_u32(smem + s * STAGE_BYTES);
+                    const uint32_t b = a + A_BYTES;
+#pragma unroll
+                    for (int ks = 0; ks < BK / 16; ++ks)
+                        mma_bf16(d, sdesc(a + ks * 32, 16, 1024), sdesc(b + ks * 2048, 8192, 1024),
+                                 idesc, (kb | ks) ? 1u : 0u);
+                    any = true;
+                    mma_commit(&empty[s]);
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1;
+                    }
+                }
+                if (!ok) break;
+                mma_commit(&tfull[acc]);
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_ph ^= 1;
+                }
+            }
+            if (abort_flag && any) {  // let every issued MMA finish before TMEM goes
+                mma_commit(drain);
+                mbar_drain(drain, 0, p.wait_ns);
+            }
+        }
+    } else {  // epilogue: warp w reads TMEM lanes 32*(w % 4) .. +31
+        const int q = warp & 3;
+        int acc = 0;
+        uint32_t acc_ph = 0;
+        for (int tile = blockIdx.x; tile < total && !abort_flag; tile += gridDim.x) {
+            int pair, mt, nt, r, g;
+            locate(tile, pair, mt, nt);
+            pair_rg(pair, r, g);
+            const int glo = g ? __ldg(p.cu + r * G + g - 1) : 0;
+            const int ghi = __ldg(p.cu + r * G + g);
+            uint64_t* bar = p.debug_stall ? never : &tfull[acc];
+            if (!mbar_wait(bar, acc_ph, p.wait_ns, &abort_flag)) break;
+            asm volatile("tcgen05.fence::after_thread_sync;");
+            const int row_in = mt * BM + q * 32 + lane;
+            const bool valid = glo + row_in < ghi;
+            uint16_t* yrow = p.y + (size_t)(r * p.C + glo + row_in) * p.Hp + nt * BN;
+            const uint32_t tbase = tmem + acc * BN + ((uint32_t)(q * 32) << 16);
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                uint32_t v[32];
+                asm volatile(
+                    "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,"
+                    "%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,"
+                    "%31}, [%32];"
+                    : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+                      "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]),
+                      "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]),
+                      "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
+                      "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]),
+                      "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+                    : "r"(tbase + c0));
+                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                if (valid) {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 8) {
+                        uint4 o;
+                        o.x = pack_bf16x2(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+                        o.y = pack_bf16x2(__uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+                        o.z = pack_bf16x2(__uint_as_float(v[j + 4]), __uint_as_float(v[j + 5]));
+                        o.w = pack_bf16x2(__uint_as_float(v[j + 6]), __uint_as_float(v[j + 7]));
+                        *reinterpret_cast<uint4*>(yrow + c0 + j) = o;
+                    }
+                }
+            }
+            asm volatile("tcgen05.fence::before_thread_sync;");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[acc]);
+            if (++acc == 2) {
+                acc = 0;
+                acc_ph ^= 1;
+            }
+        }
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;");
+    __syncthreads();
+    if (warp == 1) {
+        asm volatile("tcgen05.fence::after_thread_sync;");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"(TMEM_COLS));
+    }
+    if (tid == 0 && abort_flag) atomicMax(p.status + ST_STATUS, MOONEP_STATUS_TIMEOUT);
+}
+
+using PFN_encodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                     const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                     const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                     CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+PFN_encodeTiled encoder() {
+    static PFN_encodeTiled fn = [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return (PFN_encodeTiled) nullptr;
+        return reinterpret_cast<PFN_encodeTiled>(f);
+    }();
+    return fn;
+}
+
+bool encode_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+               uint32_t box_inner, uint32_t box_outer) {
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {inner * 2};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t es[2] = {1, 1};
+    return encoder()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                     box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// alignment slack + stages + barriers (2 per stage, 2 + 2 accumulator, drain,
+// never) + TMEM address + per-warp sums + the m-tile prefix
+size_t smem_bytes(int bn, int stages, int npairs) {
+    return 1024 + (size_t)stages * (A_BYTES + BK * bn * 2) + (size_t)(2 * stages + 6) * 8 + 8 +
+           8 * 4 + (size_t)(npairs + 1) * 4;
+}
+
+template <int BN, int STAGES>
+cudaError_t launch_variant(const CUtensorMap& x, const CUtensorMap& w, const GemmArgs& a,
+                           size_t smem, int grid, cudaStream_t s) {
+    static std::mutex mu;
+    static size_t set[64] = {};  // attribute value set so far, per device
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (dev < 0 || dev >= 64 || set[dev] < smem) {
+            e = cudaFuncSetAttribute(expert_gemm_kernel<BN, STAGES>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+            if (dev >= 0 && dev < 64) set[dev] = smem;
+        }
+    }
+    expert_gemm_kernel<BN, STAGES><<<grid, THREADS, smem, s>>>(x, w, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+int expert_gemm_npairs(const moonep_config& c) { return c.R * (c.E / c.R + c.B); }
+
+bool expert_gemm_fits(const moonep_config& c) {
+    return smem_bytes(128, 3, expert_gemm_npairs(c)) <= (size_t)SMEM_LIMIT;
+}
+
+cudaError_t launch_expert_gemm(const moonep_config& c, const moonep_plan_t& p, const void* x,
+                               const void* w, void* y, cudaStream_t s, const char** why) {
+    if (!encoder()) {
+        *why = "cuTensorMapEncodeTiled is unavailable";
+        return cudaErrorNotSupported;
+    }
+    const int C = c.S * c.K;
+    CUtensorMap tx, tw;
+    if (!encode_2d(&tx, x, (uint64_t)c.H, (uint64_t)c.R * C, BK, BM) ||
+        !encode_2d(&tw, w, (uint64_t)c.Hp, (uint64_t)c.R * (c.E + c.B) * c.H, 64, BK)) {
+        *why = "cuTensorMapEncodeTiled rejected the recv or weight layout";
+        return cudaErrorInvalidValue;
+    }
+    GemmArgs a;
+    a.R = c.R; a.C = C; a.E = c.E; a.B = c.B; a.Er = c.E / c.R; a.H = c.H; a.Hp = c.Hp;
+    a.cu = p.cu_seqlens;
+    a.status = p.status;
+    a.y = static_cast<uint16_t*>(y);
+    a.wait_ns = current_wait_limit_ns();
+    a.debug_stall = current_barrier_extra() != 0;
+    const int np = expert_gemm_npairs(c);
+    const int grid = device_sm_count();
+    if (c.Hp % 256 == 0) {
+        if (smem_bytes(256, 4, np) <= (size_t)SMEM_LIMIT)
+            return launch_variant<256, 4>(tx, tw, a, smem_bytes(256, 4, np), grid, s);
+        if (smem_bytes(256, 3, np) <= (size_t)SMEM_LIMIT)
+            return launch_variant<256, 3>(tx, tw, a, smem_bytes(256, 3, np), grid, s);
+    }
+    if (smem_bytes(128, 6, np) <= (size_t)SMEM_LIMIT)
+        return launch_variant<128, 6>(tx, tw, a, smem_bytes(128, 6, np), grid, s);
+    return launch_variant<128, 3>(tx, tw, a, smem_bytes(128, 3, np), grid, s);
+}
+
+}  // namespace moonep

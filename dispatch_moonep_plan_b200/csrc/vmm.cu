@@ -8,6 +8,9 @@
 // is mapped at the start of every rank's view, and each rank maps its own
 // physical block of B slots behind it.  Every view is contiguous, a home
 // expert exists once in memory, and a slot write is private to its rank.
+// The R views are reserved as one address range, view r at r * view_bytes,
+// so that a consumer can address all of them from one base pointer (the
+// grouped expert GEMM builds a single TMA tensor map over them).
 //
 // The driver's virtual-memory calls are taken through cudaGetDriverEntryPoint
 // so that the library does not link against the driver library itself.
@@ -75,6 +78,7 @@ struct Impl {
     bool home_made = false;
     CUmemGenericAllocationHandle slot[MOONEP_MAX_R] = {};
     bool slot_made[MOONEP_MAX_R] = {};
+    CUdeviceptr base = 0;  // one reservation of R * view_bytes
     CUdeviceptr va[MOONEP_MAX_R] = {};
     bool home_mapped[MOONEP_MAX_R] = {};
     bool slot_mapped[MOONEP_MAX_R] = {};
@@ -85,9 +89,9 @@ void teardown(Impl* m) {
     for (int r = 0; r < m->R; ++r) {
         if (m->slot_mapped[r]) d.unmap(m->va[r] + m->home_bytes, m->slot_bytes);
         if (m->home_mapped[r]) d.unmap(m->va[r], m->home_bytes);
-        if (m->va[r]) d.free_va(m->va[r], m->view_bytes);
         if (m->slot_made[r]) d.release(m->slot[r]);
     }
+    if (m->base) d.free_va(m->base, m->view_bytes * m->R);
     if (m->home_made) d.release(m->home);
 }
 
@@ -136,17 +140,17 @@ int weights_create(const moonep_config& c, int elem_bytes, moonep_weights_t* out
 
     bool fail = d.create(&m->home, m->home_bytes, &prop, 0) != CUDA_SUCCESS;
     m->home_made = !fail;
+    if (!fail) {
+        fail = d.reserve(&m->base, m->view_bytes * c.R, gran, 0, 0) != CUDA_SUCCESS;
+        if (fail) m->base = 0;
+    }
     for (int r = 0; r < c.R && !fail; ++r) {
         if (c.B > 0) {
             fail = d.create(&m->slot[r], m->slot_bytes, &prop, 0) != CUDA_SUCCESS;
             m->slot_made[r] = !fail;
             if (fail) break;
         }
-        fail = d.reserve(&m->va[r], m->view_bytes, gran, 0, 0) != CUDA_SUCCESS;
-        if (fail) {
-            m->va[r] = 0;
-            break;
-        }
+        m->va[r] = m->base + (CUdeviceptr)r * m->view_bytes;
         fail = d.map(m->va[r], m->home_bytes, 0, m->home, 0) != CUDA_SUCCESS;
         m->home_mapped[r] = !fail;
         if (fail) break;

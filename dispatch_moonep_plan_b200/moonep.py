@@ -41,7 +41,7 @@ EXPORTS = ("moonep_version", "moonep_last_error", "moonep_sizes", "moonep_plan",
            "moonep_expert_standin", "moonep_plan_status", "moonep_weights_create",
            "moonep_weights_destroy", "moonep_set_wait_limit_ns",
            "moonep_debug_set_barrier_extra", "moonep_plan_noalloc", "moonep_combine_backward",
-           "moonep_dispatch_backward")
+           "moonep_dispatch_backward", "moonep_expert_gemm")
 
 i32, i64, sz, vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p
 
@@ -103,6 +103,7 @@ def _load():
     L.moonep_plan_noalloc.argtypes = [P(Config), vp, P(Plan), vp]
     L.moonep_combine_backward.argtypes = [P(Config), P(Plan), vp, vp, vp, vp, vp, vp]
     L.moonep_dispatch_backward.argtypes = [P(Config), P(Plan), vp, vp, vp]
+    L.moonep_expert_gemm.argtypes = [P(Config), P(Plan), vp, vp, vp, vp]
     return L
 
 
@@ -220,6 +221,15 @@ def expert_standin(cfg, bufs, recv, recv_scale, mode, out, stream=None):
     _check(lib.moonep_expert_standin(ctypes.byref(cfg), ctypes.byref(bufs.c), _ptr(recv),
                                      _ptr(recv_scale), mode, _ptr(out), _stream(stream)),
            "moonep_expert_standin")
+
+
+def expert_gemm(cfg, bufs, recv, weights, out, stream=None):
+    """out[rows of group g of rank r] = recv[rows] @ weights[r][g]; ``weights``
+    is the base of R consecutive [E+B, H, Hp] bf16 views (a tensor, a
+    WeightViews' first view pointer, or an int address)."""
+    w = weights.data_ptr() if hasattr(weights, "data_ptr") else weights
+    _check(lib.moonep_expert_gemm(ctypes.byref(cfg), ctypes.byref(bufs.c), _ptr(recv), w,
+                                  _ptr(out), _stream(stream)), "moonep_expert_gemm")
 
 
 def _ptr_array(views):

@@ -270,6 +270,31 @@ int moonep_expert_standin(const moonep_config* cfg, const moonep_plan_t* plan, c
                           const float* recv_scale, int32_t mode, void* out,
                           moonep_stream_t stream);
 
+/* Grouped expert GEMM over the dispatched rows: the consumer that the pages
+ * place after dispatch, a grouped GEMM that reads the contiguous [E+B, H, H']
+ * weight tensor and selects each group's rows through cu_seqlens[E+B]
+ * ([ainovat], the framework-contract paragraph; [blog] "What This Does").
+ *
+ * recv:    bf16 [R*C, H], rank r's rows at r*C (moonep_dispatch output).
+ * weights: bf16, R consecutive [E+B, H, Hp] views; view r starts at element
+ *          r*(E+B)*H*Hp.  Row e < E of a view is home expert e, row E+j is
+ *          the replica in rank r's slot j.  The views of
+ *          moonep_weights_create(cfg, 2, &w) are laid out this way: pass
+ *          w.rank_view[0].
+ * out:     bf16 [R*C, Hp].
+ * For every rank r and group g, each row i of [cu[r][g-1], cu[r][g]) gets
+ *   out[r*C+i][:] = bf16( sum_h recv[r*C+i][h] * weights[r][g][h][:] ),
+ * products and sums in fp32 on the tensor cores (summation order not
+ * specified), then one round-to-nearest-even to bf16.  Rows of no group do
+ * not exist (every rank holds exactly C rows); only the groups a plan can
+ * fill are read: rank r's E/R home experts and its B slots.
+ * Requires payload MOONEP_PAYLOAD_BF16, H % 64 == 0, Hp % 128 == 0,
+ * R*(E+B)*H < 2^31 and 16-byte aligned pointers (else INVALID_ARG).  Does
+ * nothing when the plan's status is not OK; a device wait that runs out sets
+ * MOONEP_STATUS_TIMEOUT (out is then partly written). */
+int moonep_expert_gemm(const moonep_config* cfg, const moonep_plan_t* plan, const void* recv,
+                       const void* weights, void* out, moonep_stream_t stream);
+
 /* Wait for `stream`, then copy the first four status words to the host array
  * out[4]: status, failing rank, slots it needs, max_e T_e. */
 int moonep_plan_status(const moonep_plan_t* plan, moonep_stream_t stream, int32_t* out);
@@ -277,7 +302,8 @@ int moonep_plan_status(const moonep_plan_t* plan, moonep_stream_t stream, int32_
 /* Build R contiguous [E+B, H, Hp] views of one projection with CUDA virtual
  * memory on the current device: rows 0..E-1 of every view map the same
  * physical home block (so a home expert has one copy), rows E..E+B-1 map a
- * private slot block per rank.  This is the one-GPU form of the pages'
+ * private slot block per rank.  The views are consecutive in one address
+ * range: rank_view[r] = rank_view[0] + r*view_bytes.  This is the one-GPU form of the pages'
  * symmetric-memory weight tensor ([ainovat], the contract paragraph).
  * Requires H*Hp*elem_bytes to be a multiple of the allocation granularity
  * (2 MiB on current GPUs).  Contents are undefined until written.
@@ -317,7 +343,9 @@ int moonep_set_wait_limit_ns(uint64_t ns);
 
 /* Test hook: the planner's first grid-wide wait expects `extra` more
  * arrivals than there are blocks, so it runs out after the wait limit and
- * the plan reports MOONEP_STATUS_TIMEOUT.  0 (the default) disables it. */
+ * the plan reports MOONEP_STATUS_TIMEOUT; moonep_expert_gemm's epilogue
+ * waits on a barrier that nothing completes, with the same outcome.  0 (the
+ * default) disables it. */
 int moonep_debug_set_barrier_extra(int32_t extra);
 
 #ifdef __cplusplus
