@@ -357,6 +357,7 @@ def run_gpu(args, cfgd, emit=True):
     if emit and not args.no_side:
         out["backward"] = measure_backward(me, cfg, bufs, T, P, H, K, flush, world)
         out["side"] = measure_side(me, wl, flush, world)
+        out["expert_gemm"] = measure_gemm(me, wl, flush, world, local=local)
     if rank == 0 and emit and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline(cfgd, idx_np, w_np, x, args.rule)
         out["cpu_baseline"] = cb
@@ -554,6 +555,72 @@ def measure_side(me, wl, flush, world, reps=10):
     return out
 
 
+def tensor_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return float(d["bf16_tflops"]), float(d["bf16_tflops_sustained"]), "measured"
+    return 1590.0, 1400.0, "fallback"
+
+
+def measure_gemm(me, wl, flush, world, reps=5, S=None, local=None, rule=0):
+    """The grouped expert GEMM that consumes the plan, at the fp8 workload's
+    sizes with a bf16 payload (R16 S16384 E128 K8 H4096 B8, H'=1536): recv
+    [R*C, H] bf16, VMM-aliased [E+B, H, H'] weight views filled by the
+    replica prefetch, out [R*C, H'] bf16.  2*R*C*H*H' FLOPs per launch."""
+    import torch
+    cfgd = wl.cfg_with("fp8", payload="bf16", **({"S": S} if S else {}))
+    cfg = me.config_from(cfgd, rule)
+    idx, _ = wl.routing(cfgd, seed=0)
+    bufs = me.PlanBuffers(cfg)
+    me.plan(cfg, torch.from_numpy(idx).cuda(), bufs)
+    torch.cuda.synchronize()
+    st = me.plan_status(bufs)
+    if st[0] != me.STATUS_OK:
+        return dict(failed="plan status %s (rule %d)" % (st, rule))
+    R, E, H, Hp = cfg.R, cfg.E, cfg.H, cfg.Hp
+    P = R * cfg.S * cfg.K
+    recv = wl.hidden(P, H, seed=1, device="cuda")
+    y = torch.empty((P, Hp), dtype=torch.bfloat16, device="cuda")
+    views = me.WeightViews(cfg, elem_bytes=2)
+    try:
+        v0 = me.weight_view_tensor(views, 0, cfg, torch.bfloat16)
+        v0[:E].normal_().mul_(H ** -0.5)
+        me.prefetch(cfg, bufs, views.ptrs, 2)
+        del v0
+        stream = torch.cuda.current_stream()
+        for _ in range(3):
+            me.expert_gemm(cfg, bufs, recv, views.ptrs[0], y, stream)
+        torch.cuda.synchronize()
+        ts = []
+        with ClockSampler(local if local is not None else torch.cuda.current_device()) as clk:
+            for _ in range(reps):
+                flush()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                me.expert_gemm(cfg, bufs, recv, views.ptrs[0], y, stream)
+                b.record(stream)
+                torch.cuda.synchronize()
+                ts.append(a.elapsed_time(b))
+        st = me.plan_status(bufs)
+        if st[0] != me.STATUS_OK:
+            return dict(failed="gemm status %s" % st)
+    finally:
+        views.close()
+    t = reduce_max([statistics.mean(ts)], world)[0]
+    flops = 2.0 * P * H * Hp
+    tf = flops / (t * 1e-3) / 1e12
+    burst, sustained, kind = tensor_peaks()
+    del recv, y
+    torch.cuda.empty_cache()
+    name = cfgd["name"].replace("-fp8", "").replace("S16384", "S%d" % cfg.S)
+    return dict(workload=name + "-bf16 H'=%d" % Hp, rows=P, rule=rule,
+                ms=t, tflops=tf, flops=flops, bound="tensor",
+                peak=burst, frac=tf / burst, peak_sustained=sustained,
+                frac_sustained=tf / sustained, peak_kind=kind, reps=reps,
+                clocks=clk.summary())
+
+
 def cpu_baseline(cfgd, idx, w, x_dev, rule, budget_s=12.0):
     """The oracle, as it stands, on a bounded sample of the same workload."""
     from dispatch_moonep_plan_b200 import workloads as wl
@@ -585,6 +652,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-side", action="store_true",
                     help="skip the replica prefetch / grad-reduce measurement")
+    ap.add_argument("--gemm-only", action="store_true",
+                    help="time only the grouped expert GEMM (--S shrinks it) and print its line")
     ap.add_argument("--sweep", default=None,
                     help="also time every workload / skew and write JSON lines to this file")
     args = ap.parse_args(argv)
@@ -598,11 +667,27 @@ def main(argv=None):
     if args.impl == "reference":
         run_reference(args, cfgd)
         return
+    if args.gemm_only:
+        run_gemm_only(args)
+        return
     out = run_gpu(args, cfgd)
     if out is not None:
         print(json.dumps(out), flush=True)
     if args.sweep and out is not None:
         run_sweep(args)
+
+
+def run_gemm_only(args):
+    import torch
+    from dispatch_moonep_plan_b200 import moonep as me
+    from dispatch_moonep_plan_b200 import workloads as wl
+    flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    def flush():
+        flush_w.zero_()
+
+    out = measure_gemm(me, wl, flush, 1, reps=args.steps, S=args.S, rule=args.rule)
+    print(json.dumps(dict(expert_gemm=out)), flush=True)
 
 
 def run_sweep(args):
