@@ -117,8 +117,93 @@ __global__ void __launch_bounds__(THREADS) combine_kernel(const uint4* __restric
 // chunks in increasing position, the 8 elements of a chunk in order), then a
 // fixed xor-shuffle tree adds the 32 lane sums, so the result depends only on
 // H, not on the launch.
+// Up to 8 picks (the usual K): every lane first loads its U chunks of dy and
+// of all K expert-output rows (up to 9*U 16-byte loads in flight per lane),
+// then does the arithmetic and the K stores.  Measured against loading each
+// pick's row just before its use: 0.92-0.96 of the copy peak instead of
+// 0.72-0.74 (the loads no longer wait on one another).
 template <int U, int KMAX>
-__global__ void __launch_bounds__(THREADS) combine_bwd_kernel(const uint4* __restrict__ dy,
+__global__ void __launch_bounds__(THREADS, 2) combine_bwd_kernel(const uint4* __restrict__ dy,
+                                                             const uint4* __restrict__ eo,
+                                                             const float* __restrict__ w,
+                                                             const int32_t* __restrict__ dst_row,
+                                                             uint4* __restrict__ d_eo,
+                                                             float* __restrict__ d_w,
+                                                             const int32_t* __restrict__ status,
+                                                             int T, int K, int H8) {
+    if (load_status(status) != MOONEP_STATUS_OK) return;
+    const int lane = threadIdx.x & 31;
+    const int P = T * K;
+    const long long nw = (long long)gridDim.x * WARPS;
+    for (long long t = (long long)blockIdx.x * WARPS + (threadIdx.x >> 5); t < T; t += nw) {
+        int myrow = lane < K ? __ldg(dst_row + t * K + lane) : 0;
+        if ((unsigned)myrow >= (unsigned)P) myrow = 0;  // range guard
+        const float myw = lane < K ? __ldg(w + t * K + lane) : 0.0f;
+        long long base[KMAX];
+        float wk[KMAX];
+#pragma unroll
+        for (int k = 0; k < KMAX; ++k) {
+            base[k] = (long long)__shfl_sync(0xffffffffu, myrow, k < K ? k : 0) * H8;
+            wk[k] = __shfl_sync(0xffffffffu, myw, k < K ? k : 0);
+        }
+        float part[KMAX];
+#pragma unroll
+        for (int k = 0; k < KMAX; ++k) part[k] = 0.0f;
+        for (int c0 = 0; c0 < H8; c0 += 32 * U) {
+            uint4 gv[U];
+            uint4 ev[KMAX][U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int c = c0 + u * 32 + lane;
+                gv[u] = c < H8 ? ld_stream_v4(dy + t * H8 + c) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int k = 0; k < KMAX; ++k)
+                if (k < K)
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        const int c = c0 + u * 32 + lane;
+                        ev[k][u] = c < H8 ? ld_stream_v4(eo + base[k] + c) : make_uint4(0, 0, 0, 0);
+                    }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int c = c0 + u * 32 + lane;
+                if (c >= H8) continue;
+                const float g[8] = {bf16_lo(gv[u].x), bf16_hi(gv[u].x), bf16_lo(gv[u].y),
+                                    bf16_hi(gv[u].y), bf16_lo(gv[u].z), bf16_hi(gv[u].z),
+                                    bf16_lo(gv[u].w), bf16_hi(gv[u].w)};
+#pragma unroll
+                for (int k = 0; k < KMAX; ++k)
+                    if (k < K) {
+                        const uint4 v = ev[k][u];
+                        const float e[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                                            bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) part[k] = __fmaf_rn(g[i], e[i], part[k]);
+                        uint4 o;
+                        o.x = pack_bf16x2(__fmul_rn(wk[k], g[0]), __fmul_rn(wk[k], g[1]));
+                        o.y = pack_bf16x2(__fmul_rn(wk[k], g[2]), __fmul_rn(wk[k], g[3]));
+                        o.z = pack_bf16x2(__fmul_rn(wk[k], g[4]), __fmul_rn(wk[k], g[5]));
+                        o.w = pack_bf16x2(__fmul_rn(wk[k], g[6]), __fmul_rn(wk[k], g[7]));
+                        st_stream_v4(d_eo + base[k] + c, o);
+                    }
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < KMAX; ++k) {
+            if (k < K) {
+                float v = part[k];
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+                if (lane == 0) d_w[t * K + k] = v;
+            }
+        }
+    }
+}
+
+// More than 8 picks: the same arithmetic, one pick's row loaded at a time.
+template <int U, int KMAX>
+__global__ void __launch_bounds__(THREADS) combine_bwd_seq_kernel(const uint4* __restrict__ dy,
                                                              const uint4* __restrict__ eo,
                                                              const float* __restrict__ w,
                                                              const int32_t* __restrict__ dst_row,
@@ -223,15 +308,21 @@ cudaError_t launch_combine_backward(const moonep_config& c, const moonep_plan_t&
     const uint4* eo4 = (const uint4*)eo;
     uint4* de4 = (uint4*)d_eo;
     if (c.K <= 8) {
+        // about 128 registers: 2 blocks resident per SM; an oversubscribed
+        // grid of 8 blocks per SM measured best (0.93 at H 2048, 0.94 at 7168)
+        const int sms = device_sm_count();
+        long long g8 = ((long long)T + WARPS - 1) / WARPS;
+        if (g8 > (long long)sms * 8) g8 = (long long)sms * 8;
         if (H8 >= 64)
-            combine_bwd_kernel<2, 8><<<grid, THREADS, 0, s>>>(dy4, eo4, w, p.dst_row, de4, d_w,
-                                                             p.status, T, c.K, H8);
+            combine_bwd_kernel<2, 8><<<(int)g8, THREADS, 0, s>>>(dy4, eo4, w, p.dst_row, de4, d_w,
+                                                                p.status, T, c.K, H8);
         else
-            combine_bwd_kernel<1, 8><<<grid, THREADS, 0, s>>>(dy4, eo4, w, p.dst_row, de4, d_w,
-                                                             p.status, T, c.K, H8);
+            combine_bwd_kernel<1, 8><<<(int)g8, THREADS, 0, s>>>(dy4, eo4, w, p.dst_row, de4, d_w,
+                                                                p.status, T, c.K, H8);
     } else {
-        combine_bwd_kernel<1, MOONEP_MAX_K><<<grid, THREADS, 0, s>>>(dy4, eo4, w, p.dst_row, de4,
-                                                                    d_w, p.status, T, c.K, H8);
+        combine_bwd_seq_kernel<1, MOONEP_MAX_K><<<grid, THREADS, 0, s>>>(dy4, eo4, w, p.dst_row,
+                                                                        de4, d_w, p.status, T, c.K,
+                                                                        H8);
     }
     return cudaGetLastError();
 }
