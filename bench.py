@@ -165,24 +165,53 @@ def rank_seed(base, rank):
 
 
 # ---------------------------------------------------------------- oracle arm
-def oracle_step_estimate(cfgd, idx, w, x_bits, rule, n_tokens, rng_seed=0):
-    """One oracle step: the full plan, then dispatch + stand-in expert +
-    combine for n sampled tokens, extrapolated to all T tokens.  Returns
-    (seconds for a full step, plan seconds, sample seconds)."""
+def oracle_step_estimate(cfgd, idx, w, x_bits, rule, n_tokens, rng_seed=0, parts=None):
+    """One oracle step: the full plan, then dispatch, the identity stand-in
+    expert and combine for n sampled tokens, each timed and extrapolated to
+    all T tokens.  Returns (seconds for a full step, plan seconds, sample
+    seconds); `parts`, if given, receives the extrapolated seconds per step."""
     import numpy as np
 
     import oracle
     R, S, E, K, B = (cfgd[k] for k in ("R", "S", "E", "K", "B"))
-    T = R * S
+    T, C = R * S, S * K
+    fp8 = cfgd.get("payload") == "fp8"
     t0 = time.perf_counter()
     pl = oracle.plan(R, S, E, K, B, idx, rule=rule)
     t1 = time.perf_counter()
     tokens = np.random.default_rng(rng_seed).choice(T, size=min(n_tokens, T), replace=False)
-    oracle.path_tokens(cfgd, x_bits, w, pl, tokens, expert="identity",
-                       payload=cfgd.get("payload", "bf16"))
+    rows = pl["dst_row"][tokens].reshape(-1).astype(np.int64)
+    if fp8:
+        q, sc = oracle.dispatch_rows_fp8(K, x_bits, pl["src_of_row"], rows)
+    else:
+        recv = oracle.dispatch_rows(K, x_bits, pl["src_of_row"], rows)
     t2 = time.perf_counter()
-    full = (t1 - t0) + (t2 - t1) * T / len(tokens)
-    return full, t1 - t0, t2 - t1
+    if fp8:
+        eo = oracle.expert_rows("identity", E, B, C, pl, rows, q=q, s=sc)
+    else:
+        eo = oracle.expert_rows("identity", E, B, C, pl, rows, recv_bits=recv)
+    t3 = time.perf_counter()
+    oracle.combine_tokens(np.asarray(w, np.float32)[tokens], eo.reshape(tokens.size, K, -1))
+    t4 = time.perf_counter()
+    scale = T / len(tokens)
+    full = (t1 - t0) + (t4 - t1) * scale
+    if parts is not None:
+        parts.update(plan_ms=(t1 - t0) * 1e3, dispatch_ms=(t2 - t1) * scale * 1e3,
+                     expert_ms=(t3 - t2) * scale * 1e3, combine_ms=(t4 - t3) * scale * 1e3)
+    return full, t1 - t0, t4 - t1
+
+
+def host_cpu():
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return dict(cpu_model=model, nproc=os.cpu_count())
 
 
 def run_reference(args, cfgd):
@@ -202,9 +231,11 @@ def run_reference(args, cfgd):
     for _ in range(args.warmup):
         oracle_step_estimate(cfgd, idx, w, x_bits, args.rule, n_tok)
     steps = []
+    parts = {}
     t0 = time.perf_counter()
     for i in range(args.steps):
-        steps.append(oracle_step_estimate(cfgd, idx, w, x_bits, args.rule, n_tok, rng_seed=i)[0])
+        steps.append(oracle_step_estimate(cfgd, idx, w, x_bits, args.rule, n_tok, rng_seed=i,
+                                          parts=parts)[0])
     wall = time.perf_counter() - t0
     step_s = statistics.mean(steps)
     value = P / step_s
@@ -215,7 +246,8 @@ def run_reference(args, cfgd):
                 steps=args.steps, warmup=args.warmup, ms_per_step=step_s * 1e3,
                 higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16",
                 data="synthetic", config=workload_config(cfgd, args),
-                cpu_baseline=dict(kind="oracle", value=value, unit=UNIT, cores=1, sample=sample),
+                cpu_baseline=dict(kind="oracle", value=value, unit=UNIT, cores=1, sample=sample,
+                                  last_step_parts=parts, **host_cpu()),
                 e2e=dict(value=value, unit=UNIT, h2d_bytes_per_step=0, d2h_bytes_per_step=0),
                 wall_s=wall)
     print(json.dumps(line), flush=True)
@@ -266,7 +298,11 @@ def run_gpu(args, cfgd, emit=True):
     flush_r = torch.zeros(FLUSH_READ_BYTES // 4, dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
 
+    warm = getattr(args, "warm_l2", False)
+
     def flush():
+        if warm:  # sweep-only: the tiny workload fits in L2 and is also timed warm
+            return
         flush_w.zero_()
         flush_r.sum()
 
@@ -314,6 +350,8 @@ def run_gpu(args, cfgd, emit=True):
     t_step = [a + b + c for a, b, c in zip(t_plan, t_disp, t_comb)]
     region_ms = region[0].elapsed_time(region[1])
     m_plan, m_disp, m_comb, m_step = (statistics.mean(v) for v in (t_plan, t_disp, t_comb, t_step))
+    med = dict(plan_us=statistics.median(t_plan) * 1e3, dispatch_us=statistics.median(t_disp) * 1e3,
+               combine_us=statistics.median(t_comb) * 1e3, step_ms=statistics.median(t_step))
     m_plan, m_disp, m_comb, m_step, region_ms = reduce_max(
         [m_plan, m_disp, m_comb, m_step, region_ms], world)
 
@@ -344,7 +382,7 @@ def run_gpu(args, cfgd, emit=True):
         dispatch_GBps=disp_gbs, combine_GBps=comb_gbs,
         dispatch_frac=disp_gbs / peak, combine_frac=comb_gbs / peak,
         maxvio=maxvio, tokens_per_s=world * T / (m_step * 1e-3),
-        region_ms=region_ms,
+        region_ms=region_ms, median=med,
         e2e=dict(value=world * P / (e2e["ms"] * 1e-3), unit=UNIT,
                  h2d_bytes_per_step=e2e["h2d"], d2h_bytes_per_step=e2e["d2h"],
                  ms_per_step=e2e["ms"], serial_ms_per_step=e2e["serial_ms"],
@@ -605,11 +643,30 @@ def measure_gemm(me, wl, flush, world, reps=5, S=None, local=None, rule=0):
         st = me.plan_status(bufs)
         if st[0] != me.STATUS_OK:
             return dict(failed="gemm status %s" % st)
+        # context: cuBLAS (torch.matmul) on the same rows, one dense [H, H']
+        # weight, same data distribution, timed the same way
+        w0 = me.weight_view_tensor(views, 0, cfg, torch.bfloat16)[0].clone()
+        for _ in range(3):
+            torch.matmul(recv, w0, out=y)
+        torch.cuda.synchronize()
+        tc = []
+        with ClockSampler(local if local is not None else torch.cuda.current_device()) as clk_c:
+            for _ in range(reps):
+                flush()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                torch.matmul(recv, w0, out=y)
+                b.record(stream)
+                torch.cuda.synchronize()
+                tc.append(a.elapsed_time(b))
+        del w0
     finally:
         views.close()
     t = reduce_max([statistics.mean(ts)], world)[0]
+    t_c = reduce_max([statistics.mean(tc)], world)[0]
     flops = 2.0 * P * H * Hp
     tf = flops / (t * 1e-3) / 1e12
+    tf_c = flops / (t_c * 1e-3) / 1e12
     burst, sustained, kind = tensor_peaks()
     del recv, y
     torch.cuda.empty_cache()
@@ -618,7 +675,11 @@ def measure_gemm(me, wl, flush, world, reps=5, S=None, local=None, rule=0):
                 ms=t, tflops=tf, flops=flops, bound="tensor",
                 peak=burst, frac=tf / burst, peak_sustained=sustained,
                 frac_sustained=tf / sustained, peak_kind=kind, reps=reps,
-                clocks=clk.summary())
+                clocks=clk.summary(),
+                cublas_same_data=dict(
+                    what="torch.matmul of the same rows by one dense [H, H'] weight (no groups), "
+                         "same data, same timing; context, not the denominator",
+                    ms=t_c, tflops=tf_c, ratio=tf / tf_c, clocks=clk_c.summary()))
 
 
 def cpu_baseline(cfgd, idx, w, x_dev, rule, budget_s=12.0):
@@ -631,11 +692,12 @@ def cpu_baseline(cfgd, idx, w, x_dev, rule, budget_s=12.0):
     # grow the sample to use about budget_s of CPU time
     per_tok = ts / n
     n2 = int(max(n, min(T, (budget_s - tp) / max(per_tok, 1e-9))))
-    full, tp, ts = oracle_step_estimate(cfgd, idx, w, x_bits, rule, n2, rng_seed=1)
+    parts = {}
+    full, tp, ts = oracle_step_estimate(cfgd, idx, w, x_bits, rule, n2, rng_seed=1, parts=parts)
     return dict(kind="oracle", value=P / full, unit=UNIT, cores=1,
                 sample="full oracle plan (%d picks, %.3f s) + dispatch/identity expert/combine "
                        "of %d of %d tokens (%.2f s), extrapolated to the whole step"
-                       % (P, tp, n2, T, ts))
+                       % (P, tp, n2, T, ts), ms_per_step=full * 1e3, **parts, **host_cpu())
 
 
 def main(argv=None):
@@ -694,16 +756,20 @@ def run_sweep(args):
     """Every workload and skew level, one JSON line each (not the headline)."""
     import torch
     from dispatch_moonep_plan_b200 import workloads as wl
-    cases = [("tiny", None, 0), ("uniform", None, 0)]
+    cases = [("tiny", None, 0), ("tiny-warm", None, 0), ("uniform", None, 0)]
     cases += [("zipf", a, r) for a in (0.0, 0.5, 1.0, 1.5) for r in (0, 1)]
-    cases += [("hot", None, 0), ("hot", None, 1), ("fp8", None, 0), ("fp8", None, 1)]
+    cases += [("hot", None, 0), ("hot", None, 1), ("hot", None, 2), ("hot_tokens", None, 0),
+              ("hot_tokens", None, 1), ("fp8", None, 0), ("fp8", None, 1), ("fp8", None, 2)]
     with open(args.sweep, "w") as f:
         for name, alpha, rule in cases:
             a = argparse.Namespace(**vars(args))
             a.alpha, a.rule, a.no_cpu_baseline, a.no_side, a.no_e2e = alpha, rule, True, True, True
             a.steps = min(args.steps, 50)
+            a.warm_l2 = name.endswith("-warm")
             try:
-                out = run_gpu(a, wl.WORKLOADS[name], emit=False)
+                out = run_gpu(a, wl.WORKLOADS[name.replace("-warm", "")], emit=False)
+                if a.warm_l2:
+                    out["config"]["l2"] = "warm: no flush between steps (the whole step fits in L2)"
             except SystemExit as e:
                 out = dict(workload=name, alpha=alpha, rule=rule, failed=str(e))
             f.write(json.dumps(out) + "\n")

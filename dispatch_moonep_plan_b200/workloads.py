@@ -17,6 +17,10 @@ Routing recipes
                 over the experts other than h, then exactly floor(P/2) seeded
                 pick positions are overwritten with h (a token may then hold h
                 more than once).
+  hot_tokens    the reading of "50% of the traffic to one expert" that keeps a
+                token's K picks distinct: every token draws K picks zipf(1.0)
+                over the experts other than a seeded hot expert h, then the
+                first pick of exactly floor(T/2) seeded tokens becomes h.
 Combine weights are the softmax of K N(0,1) logits per token unless the
 recipe says otherwise.  Hidden states are N(0,1) rounded to bf16.
 """
@@ -33,6 +37,9 @@ WORKLOADS = {
                expert="scale", payload="bf16"),
     "hot": dict(name="R32-S8192-E384-K8-H7168-hot50", R=32, S=8192, E=384, K=8, H=7168,
                B=16, Hp=0, routing="hot_half", alpha=1.0, expert="identity",
+               payload="bf16"),
+    "hot_tokens": dict(name="R32-S8192-E384-K8-H7168-hot50tok", R=32, S=8192, E=384, K=8,
+               H=7168, B=16, Hp=0, routing="hot_tokens", alpha=1.0, expert="identity",
                payload="bf16"),
     "fp8": dict(name="R16-S16384-E128-K8-H4096-zipf1.2-fp8", R=16, S=16384, E=128, K=8,
                H=4096, B=8, Hp=1536, routing="zipf", alpha=1.2, expert="identity",
@@ -95,6 +102,12 @@ def routing(cfg, seed=0, alpha=None):
         flat = idx.reshape(-1)
         pos = rng.permutation(T * K)[: (T * K) // 2]
         flat[pos] = hot
+        w = _softmax_rows(rng.standard_normal((T, K)))
+    elif kind == "hot_tokens":
+        hot = int(rng.integers(E))
+        idx = zipf_topk(rng, T, E, K, cfg["alpha"] if alpha is None else alpha, exclude=hot)
+        tok = rng.permutation(T)[: T // 2]
+        idx[tok, 0] = hot
         w = _softmax_rows(rng.standard_normal((T, K)))
     elif kind == "round_robin":
         p = np.arange(T * K, dtype=np.int64)

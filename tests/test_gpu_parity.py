@@ -160,13 +160,16 @@ def test_zipf_sweep(alpha, rule):
         assert o["status"] == 0  # keep-lightest fits the slot budget at every skew
 
 
-@pytest.mark.parametrize("rule", [0, 2])
-def test_hot_adversarial(rule):
-    cfgd = wl.WORKLOADS["hot"]
+@pytest.mark.parametrize("name,rule", [("hot", 0), ("hot", 2), ("hot_tokens", 0), ("hot_tokens", 1)])
+def test_hot_adversarial(name, rule):
+    cfgd = wl.WORKLOADS[name]
     idx, w, x = routing_and_x(cfgd, seed=0)
     out, o = _check_large(cfgd, idx, w, x, rule, "identity", n_sample=256)
     assert o["status"] == 0
-    assert o["maxvio"] > 100  # half of all picks on one expert
+    if name == "hot":
+        assert o["maxvio"] > 100  # half of all picks on one expert
+    else:
+        assert o["expert_count"].max() >= cfgd["R"] * cfgd["S"] // 2  # half the tokens
     del out
     torch.cuda.empty_cache()
 

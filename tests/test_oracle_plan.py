@@ -153,7 +153,8 @@ def test_maxvio_closed_forms(oracle_mod):
 
 
 @pytest.mark.parametrize("name,alpha", [("tiny", None), ("uniform", None), ("zipf", 0.0), ("zipf", 0.5),
-                                        ("zipf", 1.0), ("zipf", 1.5)])
+                                        ("zipf", 1.0), ("zipf", 1.5), ("hot", None),
+                                        ("hot_tokens", None), ("fp8", None)])
 @pytest.mark.parametrize("rule", [0, 1, 2])
 def test_workload_plans_invariants(oracle_mod, name, alpha, rule):
     cfg = wl.WORKLOADS[name]
