@@ -59,7 +59,10 @@ __global__ void __launch_bounds__(THREADS) combine_kernel(const uint4* __restric
     if (load_status(status) != MOONEP_STATUS_OK) return;
     const int lane = threadIdx.x & 31;
     const long long nw = (long long)gridDim.x * WARPS;
-    for (long long t = (long long)blockIdx.x * WARPS + (threadIdx.x >> 5); t < T; t += nw) {
+    for (long long i = (long long)blockIdx.x * WARPS + (threadIdx.x >> 5); i < T; i += nw) {
+        // combine takes the tokens last to first: dispatch wrote the rows of
+        // the last tokens last, so those are the rows still held in L2
+        const long long t = WEIGHTED ? T - 1 - i : i;
         int myrow = lane < K ? __ldg(dst_row + t * K + lane) : 0;
         if ((unsigned)myrow >= (unsigned)(T * K)) myrow = 0;  // range guard
         const float myw = (WEIGHTED && lane < K) ? __ldg(w + t * K + lane) : 1.0f;

@@ -23,14 +23,14 @@
 //      totals (no further grid-wide wait is needed); block 0 writes the
 //      per-layer outputs, each block writes cu_seqlens / slot_expert of the
 //      ranks it owns; then every warp walks its picks again, 32 at a time, in
-//      (t, k) order; match_any gives each pick its rank among the group's
-//      picks of the same expert.  A warp's running per-expert offsets start at
-//      the block's offset plus the counts of the block's earlier warps, so the
-//      placement is stable and deterministic without ordered atomics.  The
-//      ranking is bound by the warp-shuffle crossbar (match_any, a 32-lane
-//      bitonic sort and a shuffle loop all measure about 2000 cycles per
-//      group of 32 picks at 32 warps per SM); the positions are looked up in
-//      per-expert tables so that the rest of the walk is a few shared loads.
+//      (t, k) order; the lanes holding the same expert are found with one
+//      ballot per bit of the expert index, and a pick's rank among them is
+//      the count of lower lanes.  A warp's running per-expert offsets start
+//      at the block's offset plus the counts of the block's earlier warps, so
+//      the placement is stable and deterministic without ordered atomics.
+//      (In this kernel the ballots and match_any time the same.)  The
+//      positions are looked up in per-expert tables so that the rest of the
+//      walk is a few shared loads.
 // The wait is bounded (globaltimer); when it runs out the block records
 // MOONEP_STATUS_TIMEOUT and returns.
 #include <algorithm>
@@ -95,13 +95,14 @@ struct Smem {
 };
 
 __host__ __device__ inline size_t smem_ints(int E, int R) {
-    return (size_t)NW * E + 11 * (size_t)E + 4 * ((size_t)E + 1) + 9 * (size_t)R +
+    return (size_t)NW * E + 11 * (size_t)E + 3 + 4 * ((size_t)E + 1) + 9 * (size_t)R +
            2 * SCAN_N * 32 + 8;
 }
 
 __device__ inline Smem carve(int* base, int E, int R) {
     Smem s;
     int* p = base;
+    s.ov = p; p += (E + 3) & ~3;  // first and padded: read four at a time
     s.whist = p; p += NW * E;
     s.cnt = p; p += E;
     s.bcnt = p; p += E;
@@ -110,7 +111,6 @@ __device__ inline Smem carve(int* base, int E, int R) {
     s.nzlist = p; p += E;
     s.pc = p; p += E + 1;
     s.pk = p; p += E + 1;
-    s.ov = p; p += E;
     s.item_at = p; p += E;
     s.osi = p; p += E + 1;
     s.nzri = p; p += E + 1;
@@ -238,9 +238,17 @@ __device__ int balance(const PlanParams& p, Smem& s, int* misc) {
     int ip = e;
     if (p.rule == MOONEP_RULE_LARGEST_FIRST) {
         __syncthreads();
-        if (ve) {
+        if (ve) {  // rank by counting; four experts per (broadcast) shared load
             ip = 0;
-            for (int e2 = 0; e2 < E; ++e2) {
+            const int E4 = E & ~3;
+            for (int e2 = 0; e2 < E4; e2 += 4) {
+                const int4 o4 = *reinterpret_cast<const int4*>(s.ov + e2);
+                ip += (o4.x > o) || (o4.x == o && e2 < e);
+                ip += (o4.y > o) || (o4.y == o && e2 + 1 < e);
+                ip += (o4.z > o) || (o4.z == o && e2 + 2 < e);
+                ip += (o4.w > o) || (o4.w == o && e2 + 3 < e);
+            }
+            for (int e2 = E4; e2 < E; ++e2) {
                 const int o2 = s.ov[e2];
                 ip += (o2 > o) || (o2 == o && e2 < e);
             }
@@ -366,7 +374,7 @@ __device__ __forceinline__ int place(const PlanParams& p, const Smem& s, int e, 
 }
 
 __global__ void __launch_bounds__(THREADS, 1) plan_kernel(PlanParams p) {
-    extern __shared__ int smem_raw[];
+    extern __shared__ __align__(16) int smem_raw[];
     Smem s = carve(smem_raw, p.E, p.R);
     __shared__ int wait_flag;
     __shared__ int max_count;
@@ -546,6 +554,7 @@ __global__ void __launch_bounds__(THREADS, 1) plan_kernel(PlanParams p) {
     __syncthreads();
 
     const unsigned lt_mask = (1u << lane) - 1u;
+    const int ebits = E > 1 ? 32 - __clz(E - 1) : 0;  // bits of an expert index
     int internal = 0;
     for (long long base = wlo; base < whi; base += 32 * UNR) {
         const int nu = (int)min((long long)UNR, (whi - base + 31) / 32);  // warp-uniform
@@ -560,7 +569,14 @@ __global__ void __launch_bounds__(THREADS, 1) plan_kernel(PlanParams p) {
         for (int u = 0; u < UNR; ++u) {
             if (u < nu) {
                 const int e = ev[u];
-                const unsigned peers = __match_any_sync(0xffffffffu, e);
+                // lanes holding the same expert: one ballot per bit of the
+                // expert index; lanes without a pick (e = -1) match none
+                unsigned peers = __ballot_sync(0xffffffffu, e >= 0);
+                for (int bit = 0; bit < ebits; ++bit) {
+                    const bool set = (e >> bit) & 1;
+                    const unsigned m = __ballot_sync(0xffffffffu, set);
+                    peers &= set ? m : ~m;
+                }
                 if (e >= 0) pos[u] = wh[e] + __popc(peers & lt_mask);
                 __syncwarp();
                 if (e >= 0 && lane == __ffs(peers) - 1) wh[e] += __popc(peers);
