@@ -163,10 +163,11 @@ cudaError_t launch_dispatch(const moonep_config& c, const moonep_plan_t& p, cons
     const int H8 = c.H / 8;
     if (c.payload == MOONEP_PAYLOAD_BF16) {
         // 16 chunks per lane (16 loads in flight, 2 blocks resident per SM) and
-        // a grid of 32 blocks per SM that the block scheduler balances: measured
-        // 0.96-0.99 of the copy peak, against 0.91-0.92 for 8 chunks per lane
+        // one warp per token (a grid of up to 256 blocks per SM that the block
+        // scheduler balances): measured 0.99-1.00 of the copy peak, against
+        // 0.985-0.998 on 32 blocks per SM and 0.91-0.92 for 8 chunks per lane
         // on one resident wave of blocks.
-        const int grid = grid_for(T, 32);
+        const int grid = grid_for(T, 256);
         if (H8 >= 256)
             dispatch_bf16_kernel<16><<<grid, THREADS, 0, s>>>(
                 (const uint4*)x, (uint4*)recv, p.dst_row, p.status, T, c.K, H8);
@@ -177,18 +178,30 @@ cudaError_t launch_dispatch(const moonep_config& c, const moonep_plan_t& p, cons
             dispatch_bf16_kernel<2><<<grid, THREADS, 0, s>>>(
                 (const uint4*)x, (uint4*)recv, p.dst_row, p.status, T, c.K, H8);
     } else {
-        // two units (32 elements, 4 loads) per lane, 32 blocks per SM: 0.92 of
-        // the copy peak against 0.84 for 8 elements per lane with 8-byte stores
-        const int grid = grid_for(T, 32);
+        // four units (64 elements, 8 loads) per lane when the row has at least
+        // 2048 elements, and one warp per token (the grid covers every token,
+        // up to 256 blocks per SM, so the block scheduler balances the load):
+        // 0.956 of the copy peak at H = 4096, against 0.926 for two units on
+        // 32 blocks per SM and 0.84 for 8 elements per lane with 8-byte stores
+        const int grid = grid_for(T, 256);
         const size_t smem = (size_t)WARPS * (H8 / 16) * sizeof(float);
-        if (smem > 48 * 1024) {
-            cudaError_t e = cudaFuncSetAttribute(dispatch_fp8_kernel<2>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)smem);
-            if (e != cudaSuccess) return e;
+        if (H8 >= 256) {
+            if (smem > 48 * 1024) {
+                cudaError_t e = cudaFuncSetAttribute(
+                    dispatch_fp8_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+                if (e != cudaSuccess) return e;
+            }
+            dispatch_fp8_kernel<4><<<grid, THREADS, smem, s>>>(
+                (const uint4*)x, (uint8_t*)recv, recv_scale, p.dst_row, p.status, T, c.K, H8);
+        } else {
+            if (smem > 48 * 1024) {
+                cudaError_t e = cudaFuncSetAttribute(
+                    dispatch_fp8_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+                if (e != cudaSuccess) return e;
+            }
+            dispatch_fp8_kernel<2><<<grid, THREADS, smem, s>>>(
+                (const uint4*)x, (uint8_t*)recv, recv_scale, p.dst_row, p.status, T, c.K, H8);
         }
-        dispatch_fp8_kernel<2><<<grid, THREADS, smem, s>>>(
-            (const uint4*)x, (uint8_t*)recv, recv_scale, p.dst_row, p.status, T, c.K, H8);
     }
     return cudaGetLastError();
 }
