@@ -7,10 +7,10 @@
 // bf16 (nearest even) at the end.  The k order is fixed, so the result does
 // not depend on the launch shape.
 //
-// One warp per token (grid-stride).  Lane k < K holds dst_row[t,k] and
-// w[t,k]; each lane owns U 16-byte chunks of the row, accumulates 8 floats per
-// chunk, and the next pick's chunks are loaded while the current ones are
-// accumulated.
+// One warp per token.  Lane k < K holds dst_row[t,k] and w[t,k]; each lane
+// owns U 16-byte chunks of the row and accumulates 8 floats per chunk.  Up to
+// K = 8 a lane loads its chunks of all K rows before accumulating; above that,
+// the next pick's chunks are loaded while the current ones are accumulated.
 #include <cuda_bf16.h>
 
 #include "internal.cuh"
@@ -109,6 +109,67 @@ __global__ void __launch_bounds__(THREADS) combine_kernel(const uint4* __restric
                     o.w = pack_bf16x2(acc[u][6], acc[u][7]);
                     dst[c] = o;
                 }
+            }
+        }
+    }
+}
+
+// Up to 8 picks (the usual K): every lane first loads its U chunks of all K
+// rows (up to 8*U 16-byte loads in flight), then accumulates them in k order
+// with the same fma chain.  Measured against the double-buffered form above:
+// 1.01-1.05 of the copy peak instead of 0.91-0.98 (the loads no longer wait
+// on one another; combine reads six to eight times what it writes, so it can
+// pass a copy's 1:1 rate).
+template <int U, int KMAX, bool WEIGHTED>
+__global__ void __launch_bounds__(THREADS) combine_kfirst_kernel(const uint4* __restrict__ eo,
+                                                                const float* __restrict__ w,
+                                                                const int32_t* __restrict__ dst_row,
+                                                                uint4* __restrict__ y,
+                                                                const int32_t* __restrict__ status,
+                                                                int T, int K, int H8) {
+    if (load_status(status) != MOONEP_STATUS_OK) return;
+    const int lane = threadIdx.x & 31;
+    const long long nw = (long long)gridDim.x * WARPS;
+    for (long long i = (long long)blockIdx.x * WARPS + (threadIdx.x >> 5); i < T; i += nw) {
+        // combine takes the tokens last to first: dispatch wrote the rows of
+        // the last tokens last, so those are the rows still held in L2
+        const long long t = WEIGHTED ? T - 1 - i : i;
+        int myrow = lane < K ? __ldg(dst_row + t * K + lane) : 0;
+        if ((unsigned)myrow >= (unsigned)(T * K)) myrow = 0;  // range guard
+        const float myw = (WEIGHTED && lane < K) ? __ldg(w + t * K + lane) : 1.0f;
+        long long base[KMAX];
+        float wk[KMAX];
+#pragma unroll
+        for (int k = 0; k < KMAX; ++k) {
+            base[k] = (long long)__shfl_sync(0xffffffffu, myrow, k < K ? k : 0) * H8;
+            wk[k] = __shfl_sync(0xffffffffu, myw, k < K ? k : 0);
+        }
+        for (int c0 = 0; c0 < H8; c0 += 32 * U) {
+            uint4 ev[KMAX][U];
+#pragma unroll
+            for (int k = 0; k < KMAX; ++k)
+                if (k < K)
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        const int c = c0 + u * 32 + lane;
+                        ev[k][u] = c < H8 ? ld_stream_v4(eo + base[k] + c) : make_uint4(0, 0, 0, 0);
+                    }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int c = c0 + u * 32 + lane;
+                if (c >= H8) continue;
+                float acc[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+#pragma unroll
+                for (int k = 0; k < KMAX; ++k)
+                    if (k < K) accum<WEIGHTED>(acc, wk[k], ev[k][u]);
+                uint4 o;
+                o.x = pack_bf16x2(acc[0], acc[1]);
+                o.y = pack_bf16x2(acc[2], acc[3]);
+                o.z = pack_bf16x2(acc[4], acc[5]);
+                o.w = pack_bf16x2(acc[6], acc[7]);
+                y[t * H8 + c] = o;
             }
         }
     }
@@ -285,12 +346,28 @@ int grid_4_per_sm(long long T) {
     return (int)grid;
 }
 
+// One warp per token, up to 256 blocks per SM (about 128 registers: two
+// blocks resident; the block scheduler balances the rest).
+int grid_warp_per_token(long long T) {
+    const int sms = device_sm_count();
+    long long grid = (T + WARPS - 1) / WARPS;
+    const long long cap = (long long)sms * 256;
+    if (grid > cap) grid = cap;
+    if (grid < 1) grid = 1;
+    return (int)grid;
+}
+
 }  // namespace
 
 cudaError_t launch_dispatch_backward(const moonep_config& c, const moonep_plan_t& p,
                                      const void* d_recv, void* dx, cudaStream_t s) {
     const int T = c.R * c.S;
     const int H8 = c.H / 8;
+    if (c.K <= 8) {
+        combine_kfirst_kernel<2, 8, false><<<grid_warp_per_token(T), THREADS, 0, s>>>(
+            (const uint4*)d_recv, nullptr, p.dst_row, (uint4*)dx, p.status, T, c.K, H8);
+        return cudaGetLastError();
+    }
     const int grid = grid_4_per_sm(T);
     if (H8 >= 64)
         combine_kernel<2, false><<<grid, THREADS, 0, s>>>((const uint4*)d_recv, nullptr, p.dst_row,
@@ -334,6 +411,12 @@ cudaError_t launch_combine(const moonep_config& c, const moonep_plan_t& p, const
                            const float* w, void* y, cudaStream_t s) {
     const int T = c.R * c.S;
     const int H8 = c.H / 8;
+    if (c.K <= 8) {
+        combine_kfirst_kernel<2, 8, true><<<grid_warp_per_token(T), THREADS, 0, s>>>(
+            (const uint4*)eo, w, p.dst_row, (uint4*)y, p.status, T, c.K, H8);
+        return cudaGetLastError();
+    }
+    // more than 8 picks:
     // Two 16-byte chunks per lane (double-buffered: 4 loads in flight) keep
     // the kernel near 56 registers, so 4 blocks of 256 stay resident per SM;
     // one resident wave of blocks strides over the tokens.  Measured against
