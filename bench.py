@@ -413,6 +413,7 @@ def run_gpu(args, cfgd, emit=True):
         out["backward"] = measure_backward(me, cfg, bufs, T, P, H, K, flush, world)
         out["side"] = measure_side(me, wl, flush, world)
         out["expert_gemm"] = measure_gemm(me, wl, flush, world, local=local)
+        out["expert_gemm_fp8"] = measure_gemm_fp8(me, wl, flush, world, local=local)
     if rank == 0 and emit and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline(cfgd, idx_np, w_np, x, args.rule)
         out["cpu_baseline"] = cb
@@ -739,6 +740,79 @@ def measure_gemm(me, wl, flush, world, reps=5, S=None, local=None, rule=0):
                     ms=t_c, tflops=tf_c, ratio=tf / tf_c, clocks=clk_c.summary()))
 
 
+def measure_gemm_fp8(me, wl, flush, world, reps=5, S=None, local=None, rule=0):
+    """The grouped expert GEMM on the fp8 payload at the fp8 workload's sizes:
+    the dispatched e4m3 rows and per-128 scales are widened to bf16 inside the
+    GEMM.  Beside it, the unfused route: the identity stand-in writes the
+    bf16 rows, then the bf16 GEMM reads them."""
+    import torch
+    cfgd = wl.cfg_with("fp8", **({"S": S} if S else {}))
+    cfg = me.config_from(cfgd, rule)
+    cfg16 = me.config_from(dict(cfgd, payload="bf16"), rule)
+    idx, _ = wl.routing(cfgd, seed=0)
+    bufs = me.PlanBuffers(cfg)
+    me.plan(cfg, torch.from_numpy(idx).cuda(), bufs)
+    torch.cuda.synchronize()
+    st = me.plan_status(bufs)
+    if st[0] != me.STATUS_OK:
+        return dict(failed="plan status %s (rule %d)" % (st, rule))
+    R, E, H, Hp = cfg.R, cfg.E, cfg.H, cfg.Hp
+    T, P = R * cfg.S, R * cfg.S * cfg.K
+    x = wl.hidden(T, H, seed=1, device="cuda")
+    q = torch.empty((P, H), dtype=torch.uint8, device="cuda")
+    sc = torch.empty((P, H // 128), dtype=torch.float32, device="cuda")
+    me.dispatch(cfg, bufs, x, q, sc)
+    del x
+    y = torch.empty((P, Hp), dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def timeit(fn):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            flush()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return reduce_max([statistics.mean(ts)], world)[0]
+
+    views = me.WeightViews(cfg, elem_bytes=2)
+    try:
+        v0 = me.weight_view_tensor(views, 0, cfg, torch.bfloat16)
+        v0[:E].normal_().mul_(H ** -0.5)
+        me.prefetch(cfg, bufs, views.ptrs, 2)
+        del v0
+        with ClockSampler(local if local is not None else torch.cuda.current_device()) as clk:
+            t_fused = timeit(lambda: me.expert_gemm(cfg, bufs, q, views.ptrs[0], y, stream,
+                                                    recv_scale=sc))
+        a16 = torch.empty((P, H), dtype=torch.bfloat16, device="cuda")
+        t_standin = timeit(lambda: me.expert_standin(cfg, bufs, q, sc, me.EXPERT_IDENTITY, a16,
+                                                     stream))
+        t_gemm16 = timeit(lambda: me.expert_gemm(cfg16, bufs, a16, views.ptrs[0], y, stream))
+        del a16
+        st = me.plan_status(bufs)
+        if st[0] != me.STATUS_OK:
+            return dict(failed="gemm status %s" % st)
+    finally:
+        views.close()
+    flops = 2.0 * P * H * Hp
+    burst, sustained, kind = tensor_peaks()
+    tf = flops / (t_fused * 1e-3) / 1e12
+    del q, sc, y
+    torch.cuda.empty_cache()
+    return dict(workload=cfgd["name"] + " H'=%d" % Hp, rows=P, rule=rule, ms=t_fused, tflops=tf,
+                bound="tensor", peak=burst, frac=tf / burst, peak_sustained=sustained,
+                frac_sustained=tf / sustained, peak_kind=kind, reps=reps, clocks=clk.summary(),
+                unfused=dict(standin_ms=t_standin, bf16_gemm_ms=t_gemm16,
+                             total_ms=t_standin + t_gemm16,
+                             what="identity stand-in (fp8 -> bf16 rows in HBM) then the bf16 GEMM"))
+
+
 def cpu_baseline(cfgd, idx, w, x_dev, rule, budget_s=12.0):
     """The oracle, as it stands, on a bounded sample of the same workload."""
     from dispatch_moonep_plan_b200 import workloads as wl
@@ -772,7 +846,8 @@ def main(argv=None):
     ap.add_argument("--no-side", action="store_true",
                     help="skip the replica prefetch / grad-reduce measurement")
     ap.add_argument("--gemm-only", action="store_true",
-                    help="time only the grouped expert GEMM (--S shrinks it) and print its line")
+                    help="time only the grouped expert GEMM (--S shrinks it; --workload fp8 takes "
+                         "the fp8 payload) and print its line")
     ap.add_argument("--sweep", default=None,
                     help="also time every workload / skew and write JSON lines to this file")
     args = ap.parse_args(argv)
@@ -805,6 +880,10 @@ def run_gemm_only(args):
     def flush():
         flush_w.zero_()
 
+    if args.workload == "fp8":
+        out = measure_gemm_fp8(me, wl, flush, 1, reps=args.steps, S=args.S, rule=args.rule)
+        print(json.dumps(dict(expert_gemm_fp8=out)), flush=True)
+        return
     out = measure_gemm(me, wl, flush, 1, reps=args.steps, S=args.S, rule=args.rule)
     print(json.dumps(dict(expert_gemm=out)), flush=True)
 

@@ -241,12 +241,15 @@ int moonep_expert_standin(const moonep_config* c, const moonep_plan_t* plan, con
 }
 
 int moonep_expert_gemm(const moonep_config* c, const moonep_plan_t* plan, const void* recv,
-                       const void* weights, void* out, moonep_stream_t stream) {
+                       const float* recv_scale, const void* weights, void* out,
+                       moonep_stream_t stream) {
     const char* fn = "moonep_expert_gemm";
     if (const char* why = check_config(c)) return fail(MOONEP_ERR_INVALID_ARG, fn, why);
     if (const char* why = check_plan(c, plan)) return fail(MOONEP_ERR_INVALID_ARG, fn, why);
-    if (c->payload != MOONEP_PAYLOAD_BF16)
-        return fail(MOONEP_ERR_INVALID_ARG, fn, "the expert GEMM takes the bf16 payload only");
+    if (c->payload == MOONEP_PAYLOAD_FP8 && !recv_scale)
+        return fail(MOONEP_ERR_INVALID_ARG, fn, "fp8 payload needs recv_scale");
+    if (c->payload == MOONEP_PAYLOAD_FP8 && !aligned16(recv_scale))
+        return fail(MOONEP_ERR_INVALID_ARG, fn, "recv_scale must be 16-byte aligned");
     if (c->H % 64 != 0) return fail(MOONEP_ERR_INVALID_ARG, fn, "H must be a multiple of 64");
     if (c->Hp <= 0 || c->Hp % 128 != 0)
         return fail(MOONEP_ERR_INVALID_ARG, fn, "Hp must be a positive multiple of 128");
@@ -259,8 +262,9 @@ int moonep_expert_gemm(const moonep_config* c, const moonep_plan_t* plan, const 
     if (!moonep::expert_gemm_fits(*c))
         return fail(MOONEP_ERR_INVALID_ARG, fn, "too many (rank, group) pairs for shared memory");
     const char* why = nullptr;
-    cudaError_t e = moonep::launch_expert_gemm(*c, *plan, recv, weights, out,
-                                               static_cast<cudaStream_t>(stream), &why);
+    cudaError_t e = moonep::launch_expert_gemm(
+        *c, *plan, recv, c->payload == MOONEP_PAYLOAD_FP8 ? recv_scale : nullptr, weights, out,
+        static_cast<cudaStream_t>(stream), &why);
     if (e != cudaSuccess) return cuda_fail(fn, e, why);
     return MOONEP_OK;
 }

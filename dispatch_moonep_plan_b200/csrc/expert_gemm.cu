@@ -44,8 +44,12 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int THREADS = 192;
-constexpr int A_BYTES = BM * BK * 2;  // 16 KiB
+constexpr int A_BYTES = BM * BK * 2;   // 16 KiB of bf16 A per stage
+constexpr int A8_BYTES = BM * BK;      // 8 KiB of e4m3 A per k-block (fp8 payload)
+constexpr int A8_SLOTS = 2;            // fp8 payload: e4m3 A ring, apart from the MMA ring
+// fp8 payload: CW extra warps widen A to bf16
+template <bool FP8A, int CW>
+__host__ __device__ constexpr int threads_for() { return FP8A ? (6 + CW) * 32 : 6 * 32; }
 // dynamic shared memory a CTA may ask for: the 227 KiB opt-in limit less
 // room for the kernel's static shared variables
 constexpr int SMEM_LIMIT = 227 * 1024 - 256;
@@ -149,36 +153,66 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return (uint32_t)a | ((uint32_t)b << 16);
 }
 
+// Two e4m3 codes (low byte first) -> bf16x2 of float(code) * scale: the
+// codes widen exactly to f16 and then to f32, one binary32 product each, one
+// round to nearest even to bf16.
+__device__ __forceinline__ uint32_t widen_e4m3x2(uint32_t two_codes, float scale) {
+    uint32_t h2, r;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((unsigned short)two_codes));
+    float lo, hi;
+    asm("cvt.f32.f16 %0, %1;" : "=f"(lo) : "h"((unsigned short)(h2 & 0xffffu)));
+    asm("cvt.f32.f16 %0, %1;" : "=f"(hi) : "h"((unsigned short)(h2 >> 16)));
+    // both products at once (two binary32 multiplies, round to nearest even)
+    asm("{ .reg .b64 v, s2, pr; .reg .f32 plo, phi;\n\t"
+        "mov.b64 v, {%1, %2};\n\t"
+        "mov.b64 s2, {%3, %3};\n\t"
+        "mul.rn.f32x2 pr, v, s2;\n\t"
+        "mov.b64 {plo, phi}, pr;\n\t"
+        "cvt.rn.bf16x2.f32 %0, phi, plo; }"
+        : "=r"(r)
+        : "f"(lo), "f"(hi), "f"(scale));
+    return r;
+}
+
 struct GemmArgs {
     int R, C, E, B, Er, H, Hp;
     const int32_t* cu;  // [R][E+B] inclusive row ends
     int32_t* status;
     uint16_t* y;  // [R*C, Hp] bf16
+    const float* scale;  // fp8 payload: [R*C, H/128] per-block scales
     unsigned long long wait_ns;
     int debug_stall;  // epilogue waits on a barrier nothing completes
 };
 
-template <int BN, int STAGES>
-__global__ void __launch_bounds__(THREADS, 1)
+template <int BN, int STAGES, bool FP8A, int CW>
+__global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
     expert_gemm_kernel(const __grid_constant__ CUtensorMap tmX,
                        const __grid_constant__ CUtensorMap tmW, GemmArgs p) {
+    constexpr int THREADS = threads_for<FP8A, CW>();
     constexpr int B_BYTES = BK * BN * 2;
+    // a stage of the MMA ring: bf16 A (SW128, K-major) | B.  The fp8 payload
+    // lands in its own ring of A8_SLOTS e4m3 tiles after the stages.
     constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    constexpr int A8S = FP8A ? A8_SLOTS : 0;
     constexpr int TMEM_COLS = 2 * BN;
     // k-block of A: 128 rows x 128 B; one k-step (16 elements) = 32 B along a row.
     // k-block of B: BN/64 column chunks of 64 k-rows x 128 B (8 KiB each); one
     // k-step = 16 k-rows = 2 KiB; the next 64-column chunk is 8 KiB further.
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint64_t* full = (uint64_t*)(smem + STAGES * STAGE_BYTES);
+    uint8_t* a8ring = smem + STAGES * STAGE_BYTES;  // [A8S][A8_BYTES]
+    uint64_t* full = (uint64_t*)(a8ring + A8S * A8_BYTES);
     uint64_t* empty = full + STAGES;
-    uint64_t* tfull = empty + STAGES;
+    uint64_t* conv = empty + STAGES;    // fp8 payload: the stage's A is widened
+    uint64_t* a8full = conv + STAGES;   // fp8 payload: e4m3 tile landed [A8_SLOTS]
+    uint64_t* a8empty = a8full + A8_SLOTS;  // fp8 payload: e4m3 tile read [A8_SLOTS]
+    uint64_t* tfull = a8empty + A8_SLOTS;
     uint64_t* tempty = tfull + 2;
     uint64_t* drain = tempty + 2;
     uint64_t* never = drain + 1;
     uint32_t* tmem_slot = (uint32_t*)(never + 1);
     int* wsum = (int*)(tmem_slot + 2);  // [THREADS / 32]
-    int* pre = wsum + 8;                // [npairs + 1] m-tile prefix
+    int* pre = wsum + 16;               // [npairs + 1] m-tile prefix
     __shared__ volatile int abort_flag;
     __shared__ int plan_status;
 
@@ -199,6 +233,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
+            mbar_init(&conv[s], CW);
+        }
+        for (int j = 0; j < A8_SLOTS; ++j) {
+            mbar_init(&a8full[j], 1);
+            mbar_init(&a8empty[j], CW);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
@@ -289,10 +328,24 @@ __global__ void __launch_bounds__(THREADS, 1)
                         ok = false;
                         break;
                     }
-                    mbar_expect_tx(&full[s], STAGE_BYTES);
                     uint8_t* a = smem + s * STAGE_BYTES;
                     uint8_t* b = a + A_BYTES;
-                    tma_load_2d(a, &tmX, &full[s], kb * BK, row0);
+                    if constexpr (FP8A) {
+                        // the e4m3 tile goes to its own ring; the converters
+                        // widen it into this stage's A once it lands
+                        const int j8 = (int)(issued % A8S);
+                        const uint32_t p8 = (uint32_t)((issued / A8S) & 1);
+                        if (!mbar_wait(&a8empty[j8], p8 ^ 1, p.wait_ns, &abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_expect_tx(&a8full[j8], A8_BYTES);
+                        tma_load_2d(a8ring + j8 * A8_BYTES, &tmX, &a8full[j8], kb * BK, row0);
+                        mbar_expect_tx(&full[s], B_BYTES);
+                    } else {
+                        mbar_expect_tx(&full[s], A_BYTES + B_BYTES);
+                        tma_load_2d(a, &tmX, &full[s], kb * BK, row0);
+                    }
 #pragma unroll
                     for (int j = 0; j < BN / 64; ++j)
                         tma_load_2d(b + j * 8192, &tmW, &full[s], nt * BN + 64 * j,
@@ -310,6 +363,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                 // wait for the last STAGES of them to land before leaving
                 for (long long n = issued > STAGES ? issued - STAGES : 0; n < issued; ++n)
                     mbar_drain(&full[n % STAGES], (uint32_t)((n / STAGES) & 1), p.wait_ns);
+                if constexpr (FP8A)  // and the last e4m3 tiles
+                    for (long long n = issued > A8S ? issued - A8S : 0; n < issued; ++n)
+                        mbar_drain(&a8full[n % A8S], (uint32_t)((n / A8S) & 1), p.wait_ns);
             }
         }
     } else if (warp == 1) {
@@ -330,7 +386,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint32_t d = tmem + acc * BN;
                 bool ok = true;
                 for (int kb = 0; kb < kblocks; ++kb) {
-                    if (!mbar_wait(&full[s], ph, p.wait_ns, &abort_flag)) {
+                    // the TMA loads landed; fp8: and the converter warps have
+                    // widened A into the stage
+                    if (!mbar_wait(&full[s], ph, p.wait_ns, &abort_flag) ||
+                        (FP8A && !mbar_wait(&conv[s], ph, p.wait_ns, &abort_flag))) {
                         ok = false;
                         break;
                     }
@@ -360,7 +419,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 mbar_drain(drain, 0, p.wait_ns);
             }
         }
-    } else {  // epilogue: warp w reads TMEM lanes 32*(w % 4) .. +31
+    } else if (warp < 6) {  // epilogue: warp w reads TMEM lanes 32*(w % 4) .. +31
         const int q = warp & 3;
         int acc = 0;
         uint32_t acc_ph = 0;
@@ -412,6 +471,67 @@ __global__ void __launch_bounds__(THREADS, 1)
                 acc_ph ^= 1;
             }
         }
+    } else if constexpr (FP8A) {
+        // converters: widen each e4m3 tile (row-major, 64 B a row) into the
+        // stage's bf16 A, in the 128-byte-swizzled K-major layout the MMA reads:
+        // a = bf16(float(q) * scale), one binary32 product, round to nearest
+        // even.  A warp reads 32 consecutive 16-byte chunks (8 rows) and
+        // writes each as two 16-byte bf16 chunks at their swizzled places.
+        const int ct = tid - 6 * 32;  // 0 .. CW*32 - 1
+        const int nsc = p.H / 128;    // scales per row
+        const long long nrows = (long long)p.R * p.C;
+        int s = 0;
+        long long n = 0;  // k-blocks converted: tile n % A8S of the e4m3 ring
+        for (int tile = blockIdx.x; tile < total && !abort_flag; tile += gridDim.x) {
+            int pair, mt, nt, r, g;
+            locate(tile, pair, mt, nt);
+            pair_rg(pair, r, g);
+            const long long row0 =
+                (long long)r * p.C + (g ? __ldg(p.cu + r * G + g - 1) : 0) + mt * BM;
+            bool ok = true;
+            for (int kb = 0; kb < kblocks; ++kb) {
+                // the tile landed; the producer loaded it only after this
+                // stage's previous MMAs finished, so the stage's A is free
+                const int j8 = (int)(n % A8S);
+                if (!mbar_wait(&a8full[j8], (uint32_t)((n / A8S) & 1), p.wait_ns, &abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* a16 = smem + s * STAGE_BYTES;
+                const uint8_t* a8 = a8ring + j8 * A8_BYTES;
+#pragma unroll
+                for (int j = 0; j < (BM * BK / 16) / (CW * 32); ++j) {
+                    const int chunk = j * CW * 32 + ct;
+                    const int row = chunk >> 2, cq = chunk & 3;
+                    const uint4 v = *reinterpret_cast<const uint4*>(a8 + chunk * 16);
+                    const long long grow = row0 + row;
+                    const float sc = grow < nrows ? __ldg(p.scale + grow * nsc + (kb >> 1)) : 0.0f;
+                    uint32_t o[8];
+                    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        o[2 * q] = widen_e4m3x2(w4[q] & 0xffffu, sc);
+                        o[2 * q + 1] = widen_e4m3x2(w4[q] >> 16, sc);
+                    }
+                    const int sw = row & 7;
+                    uint8_t* dst = a16 + row * 128;
+                    *reinterpret_cast<uint4*>(dst + (((2 * cq) ^ sw) << 4)) =
+                        make_uint4(o[0], o[1], o[2], o[3]);
+                    *reinterpret_cast<uint4*>(dst + (((2 * cq + 1) ^ sw) << 4)) =
+                        make_uint4(o[4], o[5], o[6], o[7]);
+                }
+                // generic-proxy stores, read next by the tensor cores
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&conv[s]);
+                    mbar_arrive(&a8empty[j8]);
+                }
+                ++n;
+                if (++s == STAGES) s = 0;
+            }
+            if (!ok) break;
+        }
     }
     asm volatile("tcgen05.fence::before_thread_sync;");
     __syncthreads();
@@ -441,26 +561,27 @@ PFN_encodeTiled encoder() {
     return fn;
 }
 
-bool encode_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
-               uint32_t box_inner, uint32_t box_outer) {
+bool encode_2d(CUtensorMap* m, const void* base, CUtensorMapDataType type, uint64_t elem_bytes,
+               uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer,
+               CUtensorMapSwizzle swizzle) {
     const cuuint64_t dims[2] = {inner, outer};
-    const cuuint64_t strides[1] = {inner * 2};
+    const cuuint64_t strides[1] = {inner * elem_bytes};
     const cuuint32_t box[2] = {box_inner, box_outer};
     const cuuint32_t es[2] = {1, 1};
-    return encoder()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                     box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    return encoder()(m, type, 2, const_cast<void*>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// alignment slack + stages + barriers (2 per stage, 2 + 2 accumulator, drain,
-// never) + TMEM address + per-warp sums + the m-tile prefix
-size_t smem_bytes(int bn, int stages, int npairs) {
-    return 1024 + (size_t)stages * (A_BYTES + BK * bn * 2) + (size_t)(2 * stages + 6) * 8 + 8 +
-           8 * 4 + (size_t)(npairs + 1) * 4;
+// alignment slack + stages + e4m3 ring + barriers (3 per stage, 2 per e4m3
+// slot, 2 + 2 accumulator, drain, never) + TMEM address + per-warp sums +
+// the m-tile prefix
+size_t smem_bytes(int bn, int stages, int npairs, bool fp8a) {
+    return 1024 + (size_t)stages * (A_BYTES + BK * bn * 2) + (fp8a ? A8_SLOTS * A8_BYTES : 0) +
+           (size_t)(3 * stages + 2 * A8_SLOTS + 6) * 8 + 8 + 16 * 4 + (size_t)(npairs + 1) * 4;
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool FP8A, int CW = 8>
 cudaError_t launch_variant(const CUtensorMap& x, const CUtensorMap& w, const GemmArgs& a,
                            size_t smem, int grid, cudaStream_t s) {
     static std::mutex mu;
@@ -471,13 +592,13 @@ cudaError_t launch_variant(const CUtensorMap& x, const CUtensorMap& w, const Gem
     {
         std::lock_guard<std::mutex> lock(mu);
         if (dev < 0 || dev >= 64 || set[dev] < smem) {
-            e = cudaFuncSetAttribute(expert_gemm_kernel<BN, STAGES>,
+            e = cudaFuncSetAttribute(expert_gemm_kernel<BN, STAGES, FP8A, CW>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return e;
             if (dev >= 0 && dev < 64) set[dev] = smem;
         }
     }
-    expert_gemm_kernel<BN, STAGES><<<grid, THREADS, smem, s>>>(x, w, a);
+    expert_gemm_kernel<BN, STAGES, FP8A, CW><<<grid, threads_for<FP8A, CW>(), smem, s>>>(x, w, a);
     return cudaGetLastError();
 }
 
@@ -486,19 +607,28 @@ cudaError_t launch_variant(const CUtensorMap& x, const CUtensorMap& w, const Gem
 int expert_gemm_npairs(const moonep_config& c) { return c.R * (c.E / c.R + c.B); }
 
 bool expert_gemm_fits(const moonep_config& c) {
-    return smem_bytes(128, 3, expert_gemm_npairs(c)) <= (size_t)SMEM_LIMIT;
+    return smem_bytes(128, 3, expert_gemm_npairs(c), c.payload == MOONEP_PAYLOAD_FP8) <=
+           (size_t)SMEM_LIMIT;
 }
 
 cudaError_t launch_expert_gemm(const moonep_config& c, const moonep_plan_t& p, const void* x,
-                               const void* w, void* y, cudaStream_t s, const char** why) {
+                               const float* x_scale, const void* w, void* y, cudaStream_t s,
+                               const char** why) {
     if (!encoder()) {
         *why = "cuTensorMapEncodeTiled is unavailable";
         return cudaErrorNotSupported;
     }
+    const bool fp8 = c.payload == MOONEP_PAYLOAD_FP8;
     const int C = c.S * c.K;
     CUtensorMap tx, tw;
-    if (!encode_2d(&tx, x, (uint64_t)c.H, (uint64_t)c.R * C, BK, BM) ||
-        !encode_2d(&tw, w, (uint64_t)c.Hp, (uint64_t)c.R * (c.E + c.B) * c.H, 64, BK)) {
+    const bool ok_x =
+        fp8 ? encode_2d(&tx, x, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)c.H, (uint64_t)c.R * C,
+                        BK, BM, CU_TENSOR_MAP_SWIZZLE_NONE)
+            : encode_2d(&tx, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)c.H,
+                        (uint64_t)c.R * C, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!ok_x || !encode_2d(&tw, w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)c.Hp,
+                            (uint64_t)c.R * (c.E + c.B) * c.H, 64, BK,
+                            CU_TENSOR_MAP_SWIZZLE_128B)) {
         *why = "cuTensorMapEncodeTiled rejected the recv or weight layout";
         return cudaErrorInvalidValue;
     }
@@ -507,19 +637,29 @@ cudaError_t launch_expert_gemm(const moonep_config& c, const moonep_plan_t& p, c
     a.cu = p.cu_seqlens;
     a.status = p.status;
     a.y = static_cast<uint16_t*>(y);
+    a.scale = x_scale;
     a.wait_ns = current_wait_limit_ns();
     a.debug_stall = current_barrier_extra() != 0;
     const int np = expert_gemm_npairs(c);
     const int grid = device_sm_count();
-    if (c.Hp % 256 == 0) {
-        if (smem_bytes(256, 4, np) <= (size_t)SMEM_LIMIT)
-            return launch_variant<256, 4>(tx, tw, a, smem_bytes(256, 4, np), grid, s);
-        if (smem_bytes(256, 3, np) <= (size_t)SMEM_LIMIT)
-            return launch_variant<256, 3>(tx, tw, a, smem_bytes(256, 3, np), grid, s);
+    if (fp8) {
+        if (c.Hp % 256 == 0 && smem_bytes(256, 4, np, true) <= (size_t)SMEM_LIMIT)
+            return launch_variant<256, 4, true>(tx, tw, a, smem_bytes(256, 4, np, true), grid, s);
+        if (c.Hp % 256 == 0 && smem_bytes(256, 3, np, true) <= (size_t)SMEM_LIMIT)
+            return launch_variant<256, 3, true>(tx, tw, a, smem_bytes(256, 3, np, true), grid, s);
+        if (smem_bytes(128, 5, np, true) <= (size_t)SMEM_LIMIT)
+            return launch_variant<128, 5, true>(tx, tw, a, smem_bytes(128, 5, np, true), grid, s);
+        return launch_variant<128, 3, true>(tx, tw, a, smem_bytes(128, 3, np, true), grid, s);
     }
-    if (smem_bytes(128, 6, np) <= (size_t)SMEM_LIMIT)
-        return launch_variant<128, 6>(tx, tw, a, smem_bytes(128, 6, np), grid, s);
-    return launch_variant<128, 3>(tx, tw, a, smem_bytes(128, 3, np), grid, s);
+    if (c.Hp % 256 == 0) {
+        if (smem_bytes(256, 4, np, false) <= (size_t)SMEM_LIMIT)
+            return launch_variant<256, 4, false>(tx, tw, a, smem_bytes(256, 4, np, false), grid, s);
+        if (smem_bytes(256, 3, np, false) <= (size_t)SMEM_LIMIT)
+            return launch_variant<256, 3, false>(tx, tw, a, smem_bytes(256, 3, np, false), grid, s);
+    }
+    if (smem_bytes(128, 6, np, false) <= (size_t)SMEM_LIMIT)
+        return launch_variant<128, 6, false>(tx, tw, a, smem_bytes(128, 6, np, false), grid, s);
+    return launch_variant<128, 3, false>(tx, tw, a, smem_bytes(128, 3, np, false), grid, s);
 }
 
 }  // namespace moonep

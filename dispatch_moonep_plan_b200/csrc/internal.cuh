@@ -97,7 +97,8 @@ cudaError_t launch_grad_reduce(const moonep_config& c, const moonep_plan_t& p,
                                float* const* views, cudaStream_t s);
 
 cudaError_t launch_expert_gemm(const moonep_config& c, const moonep_plan_t& p, const void* x,
-                               const void* w, void* y, cudaStream_t s, const char** why);
+                               const float* x_scale, const void* w, void* y, cudaStream_t s,
+                               const char** why);
 bool expert_gemm_fits(const moonep_config& c);
 
 int device_sm_count();

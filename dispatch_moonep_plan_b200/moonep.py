@@ -103,7 +103,7 @@ def _load():
     L.moonep_plan_noalloc.argtypes = [P(Config), vp, P(Plan), vp]
     L.moonep_combine_backward.argtypes = [P(Config), P(Plan), vp, vp, vp, vp, vp, vp]
     L.moonep_dispatch_backward.argtypes = [P(Config), P(Plan), vp, vp, vp]
-    L.moonep_expert_gemm.argtypes = [P(Config), P(Plan), vp, vp, vp, vp]
+    L.moonep_expert_gemm.argtypes = [P(Config), P(Plan), vp, vp, vp, vp, vp]
     return L
 
 
@@ -223,13 +223,15 @@ def expert_standin(cfg, bufs, recv, recv_scale, mode, out, stream=None):
            "moonep_expert_standin")
 
 
-def expert_gemm(cfg, bufs, recv, weights, out, stream=None):
+def expert_gemm(cfg, bufs, recv, weights, out, stream=None, recv_scale=None):
     """out[rows of group g of rank r] = recv[rows] @ weights[r][g]; ``weights``
     is the base of R consecutive [E+B, H, Hp] bf16 views (a tensor, a
-    WeightViews' first view pointer, or an int address)."""
+    WeightViews' first view pointer, or an int address).  For the fp8
+    payload, recv holds e4m3 codes and recv_scale their per-128 scales."""
     w = weights.data_ptr() if hasattr(weights, "data_ptr") else weights
-    _check(lib.moonep_expert_gemm(ctypes.byref(cfg), ctypes.byref(bufs.c), _ptr(recv), w,
-                                  _ptr(out), _stream(stream)), "moonep_expert_gemm")
+    _check(lib.moonep_expert_gemm(ctypes.byref(cfg), ctypes.byref(bufs.c), _ptr(recv),
+                                  _ptr(recv_scale), w, _ptr(out), _stream(stream)),
+           "moonep_expert_gemm")
 
 
 def _ptr_array(views):

@@ -275,7 +275,12 @@ int moonep_expert_standin(const moonep_config* cfg, const moonep_plan_t* plan, c
  * weight tensor and selects each group's rows through cu_seqlens[E+B]
  * ([ainovat], the framework-contract paragraph; [blog] "What This Does").
  *
- * recv:    bf16 [R*C, H], rank r's rows at r*C (moonep_dispatch output).
+ * recv:    the dispatched rows [R*C, H], rank r's rows at r*C
+ *          (moonep_dispatch output): bf16, or for the fp8 payload e4m3 codes
+ *          with recv_scale fp32 [R*C, H/128] (NULL for bf16).  fp8 rows are
+ *          widened in shared memory to a = bf16(float(q) * scale), one
+ *          binary32 product, round to nearest even -- the same values the
+ *          identity stand-in expert produces -- and then multiplied as bf16.
  * weights: bf16, R consecutive [E+B, H, Hp] views; view r starts at element
  *          r*(E+B)*H*Hp.  Row e < E of a view is home expert e, row E+j is
  *          the replica in rank r's slot j.  The views of
@@ -288,12 +293,13 @@ int moonep_expert_standin(const moonep_config* cfg, const moonep_plan_t* plan, c
  * specified), then one round-to-nearest-even to bf16.  Rows of no group do
  * not exist (every rank holds exactly C rows); only the groups a plan can
  * fill are read: rank r's E/R home experts and its B slots.
- * Requires payload MOONEP_PAYLOAD_BF16, H % 64 == 0, Hp % 128 == 0,
- * R*(E+B)*H < 2^31 and 16-byte aligned pointers (else INVALID_ARG).  Does
+ * Requires H % 64 == 0, Hp % 128 == 0, R*(E+B)*H < 2^31, recv_scale for
+ * the fp8 payload and 16-byte aligned pointers (else INVALID_ARG).  Does
  * nothing when the plan's status is not OK; a device wait that runs out sets
  * MOONEP_STATUS_TIMEOUT (out is then partly written). */
 int moonep_expert_gemm(const moonep_config* cfg, const moonep_plan_t* plan, const void* recv,
-                       const void* weights, void* out, moonep_stream_t stream);
+                       const float* recv_scale, const void* weights, void* out,
+                       moonep_stream_t stream);
 
 /* Wait for `stream`, then copy the first four status words to the host array
  * out[4]: status, failing rank, slots it needs, max_e T_e. */

@@ -304,5 +304,91 @@ def test_invalid_arguments_rejected_before_launch():
     with pytest.raises(m.MoonEPError, match="multiple of 128"):
         m.expert_gemm(cfg, m.PlanBuffers(cfg), x, w, y)
     cfg = m.config(2, 8, 4, 2, 2, 128, Hp=128, payload=m.PAYLOAD_FP8)
-    with pytest.raises(m.MoonEPError, match="bf16"):
+    with pytest.raises(m.MoonEPError, match="recv_scale"):
         m.expert_gemm(cfg, m.PlanBuffers(cfg), x, w, y)
+
+
+# ---------------------------------------------------------------- fp8 payload
+# e4m3 codes of the integers -2..2 (sign bit 0x80; 1.0 = 0x38, 2.0 = 0x40)
+_INT_CODES = np.array([0xC0, 0xB8, 0x00, 0x38, 0x40], np.uint8)
+
+
+def _gen_fp8(P, H, seed, integer):
+    """Seeded e4m3 rows and per-128 scales.  Integer mode: values -2..2 with
+    power-of-two scales, so every dequantised value and partial sum is exact.
+    Otherwise: any finite code and scales in [2^-8, 2^-4)."""
+    rng = np.random.default_rng(1_234 + seed)
+    if integer:
+        q = _INT_CODES[rng.integers(0, 5, (P, H))]
+        sc = (2.0 ** rng.integers(-1, 2, (P, H // 128))).astype(np.float32)
+    else:
+        q = rng.integers(0, 256, (P, H), dtype=np.uint8)
+        q[(q & 0x7F) == 0x7F] = 0x3C  # no NaN codes
+        sc = (2.0 ** rng.uniform(-8, -4, (P, H // 128))).astype(np.float32)
+    return q, sc
+
+
+def _run_fp8(cfgd, rule=1, seed=0, integer=False):
+    m = me()
+    cfgd = dict(cfgd, payload="fp8")
+    cfg, bufs, o = _plan(cfgd, rule, seed)
+    if o["status"] != 0:
+        return None
+    P, H = cfg.R * cfg.S * cfg.K, cfg.H
+    q, sc = _gen_fp8(P, H, seed, integer)
+    q_d, sc_d = torch.from_numpy(q).cuda(), torch.from_numpy(sc).cuda()
+    home = _gen((cfg.E, H, cfg.Hp), seed + 1, integer, scale=H ** -0.5)
+    w = _plain_weights(cfg, o, home)
+    y = torch.zeros((P, cfg.Hp), dtype=torch.bfloat16, device="cuda")
+    m.expert_gemm(cfg, bufs, q_d, w, y, recv_scale=sc_d)
+    torch.cuda.synchronize()
+    assert m.plan_status(bufs)[0] == m.STATUS_OK
+    # oracle: the dequantised rows (the identity stand-in's values), then the GEMM
+    C = cfg.S * cfg.K
+    rows = np.arange(P)
+    ranks, groups = oracle.row_groups(cfg.E, cfg.B, C, o["cu_seqlens"], rows)
+    experts = _experts_of(cfg, o, ranks, groups)
+    uniq, mat = np.unique(experts, return_inverse=True)
+    a_bits = oracle.dequant_rows(q, sc)
+    ref = oracle.expert_gemm_rows(a_bits, mat.astype(np.int32),
+                                  bits16(home[torch.from_numpy(uniq).cuda()]))
+    _check(bits16(y), ref, H, integer)
+    # the fused path equals the stand-in followed by the bf16 GEMM, bit for bit
+    a_dev = torch.zeros((P, H), dtype=torch.bfloat16, device="cuda")
+    m.expert_standin(cfg, bufs, q_d, sc_d, m.EXPERT_IDENTITY, a_dev)
+    cfg16 = m.config_from(dict(cfgd, payload="bf16"), rule)
+    y16 = torch.zeros_like(y)
+    m.expert_gemm(cfg16, bufs, a_dev, w, y16)
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int16), y16.view(torch.int16))
+    return dict(cfg=cfg, y=y)
+
+
+@pytest.mark.parametrize("shape", [
+    (2, 100, 4, 2, 2, 128, 256),     # BN 256, two k-blocks
+    (3, 150, 6, 2, 3, 256, 384),     # Hp 384: BN 128
+    (4, 96, 8, 3, 4, 384, 512),      # odd number of 128-blocks per row
+    (1, 300, 4, 2, 0, 128, 128),     # one rank, no slots
+])
+@pytest.mark.parametrize("integer", [True, False])
+def test_fp8_small_full(shape, integer):
+    R, S, E, K, B, H, Hp = shape
+    done = 0
+    for seed in range(2):
+        for rule in (0, 1, 2):
+            if _run_fp8(_small(R, S, E, K, B, H, Hp, alpha=1.2), rule=rule, seed=seed,
+                        integer=integer) is not None:
+                done += 1
+    assert done >= 2
+
+
+def test_fp8_random_shapes_and_ragged():
+    rng = np.random.default_rng(17)
+    done = 0
+    for it in range(8):
+        c = wl.random_small_cfg(rng, H=128 * int(rng.integers(1, 4)))
+        c["B"] = 16
+        c["Hp"] = 128 * int(rng.integers(1, 4))
+        if _run_fp8(c, rule=int(rng.integers(0, 3)), seed=it, integer=bool(it % 2)) is not None:
+            done += 1
+    assert done >= 5
