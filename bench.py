@@ -805,7 +805,8 @@ def measure_gemm_fp8(me, wl, flush, world, reps=5, S=None, local=None, rule=0):
     tf = flops / (t_fused * 1e-3) / 1e12
     del q, sc, y
     torch.cuda.empty_cache()
-    return dict(workload=cfgd["name"] + " H'=%d" % Hp, rows=P, rule=rule, ms=t_fused, tflops=tf,
+    name = cfgd["name"].replace("S16384", "S%d" % cfg.S)
+    return dict(workload=name + " H'=%d" % Hp, rows=P, rule=rule, ms=t_fused, tflops=tf,
                 bound="tensor", peak=burst, frac=tf / burst, peak_sustained=sustained,
                 frac_sustained=tf / sustained, peak_kind=kind, reps=reps, clocks=clk.summary(),
                 unfused=dict(standin_ms=t_standin, bf16_gemm_ms=t_gemm16,
