@@ -659,13 +659,19 @@ def tensor_peaks():
     return 1590.0, 1400.0, "fallback"
 
 
-def measure_gemm(me, wl, flush, world, reps=5, S=None, local=None, rule=0):
-    """The grouped expert GEMM that consumes the plan, at the fp8 workload's
-    sizes with a bf16 payload (R16 S16384 E128 K8 H4096 B8, H'=1536): recv
-    [R*C, H] bf16, VMM-aliased [E+B, H, H'] weight views filled by the
-    replica prefetch, out [R*C, H'] bf16.  2*R*C*H*H' FLOPs per launch."""
+def measure_gemm(me, wl, flush, world, reps=5, S=None, local=None, rule=0, base="fp8", Hp=None):
+    """The grouped expert GEMM that consumes the plan, by default at the fp8
+    workload's sizes with a bf16 payload (R16 S16384 E128 K8 H4096 B8,
+    H'=1536): recv [R*C, H] bf16, VMM-aliased [E+B, H, H'] weight views
+    filled by the replica prefetch, out [R*C, H'] bf16.  2*R*C*H*H' FLOPs per
+    launch.  `base` and `Hp` pick another workload's routing and sizes."""
     import torch
-    cfgd = wl.cfg_with("fp8", payload="bf16", **({"S": S} if S else {}))
+    kw = {"payload": "bf16"}
+    if S:
+        kw["S"] = S
+    if Hp or not wl.WORKLOADS[base]["Hp"]:
+        kw["Hp"] = Hp or 1536
+    cfgd = wl.cfg_with(base, **kw)
     cfg = me.config_from(cfgd, rule)
     idx, _ = wl.routing(cfgd, seed=0)
     bufs = me.PlanBuffers(cfg)
@@ -728,7 +734,7 @@ def measure_gemm(me, wl, flush, world, reps=5, S=None, local=None, rule=0):
     burst, sustained, kind = tensor_peaks()
     del recv, y
     torch.cuda.empty_cache()
-    name = cfgd["name"].replace("-fp8", "").replace("S16384", "S%d" % cfg.S)
+    name = cfgd["name"].replace("-fp8", "").replace("S%d" % wl.WORKLOADS[base]["S"], "S%d" % cfg.S)
     return dict(workload=name + "-bf16 H'=%d" % Hp, rows=P, rule=rule,
                 ms=t, tflops=tf, flops=flops, bound="tensor",
                 peak=burst, frac=tf / burst, peak_sustained=sustained,
@@ -843,6 +849,9 @@ def main(argv=None):
     ap.add_argument("--S", type=int, default=None,
                     help="tokens per rank, overriding the workload's (for small profiling cases)")
     ap.add_argument("--rule", type=int, default=0)
+    ap.add_argument("--Hp", type=int, default=None,
+                    help="with --gemm-only: the expert output width H' (default: the workload's, "
+                         "else 1536)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-side", action="store_true",
                     help="skip the replica prefetch / grad-reduce measurement")
@@ -885,7 +894,9 @@ def run_gemm_only(args):
         out = measure_gemm_fp8(me, wl, flush, 1, reps=args.steps, S=args.S, rule=args.rule)
         print(json.dumps(dict(expert_gemm_fp8=out)), flush=True)
         return
-    out = measure_gemm(me, wl, flush, 1, reps=args.steps, S=args.S, rule=args.rule)
+    base = "fp8" if args.workload == "uniform" else args.workload  # the default: fp8's sizes
+    out = measure_gemm(me, wl, flush, 1, reps=args.steps, S=args.S, rule=args.rule, base=base,
+                       Hp=args.Hp)
     print(json.dumps(dict(expert_gemm=out)), flush=True)
 
 
