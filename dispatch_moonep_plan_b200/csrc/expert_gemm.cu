@@ -10,8 +10,10 @@
 // "What This Does").  The pages give no kernel for it; this one is written
 // for sm_100a:
 //
-//  - one persistent CTA per SM, 192 threads: warp 0 issues TMA loads, one
-//    thread of warp 1 issues tcgen05.mma, warps 2-5 drain the accumulator;
+//  - one persistent CTA per SM: warp 0 issues TMA loads, one thread of warp 1
+//    issues tcgen05.mma, warps 2-5 drain the accumulator (192 threads); for
+//    the fp8 payload CW more warps widen the e4m3 rows to bf16 in shared
+//    memory (a = bf16(float(q) * scale)) between the TMA and the MMA;
 //  - tile 128 rows x BN columns (BN = 256 when H' allows, else 128), k-block
 //    64: A = 128 x 64 bf16 rows of the dispatched block (K-major), B = 64 x BN
 //    of the weight row (H' contiguous, MN-major), both 128-byte swizzled;

@@ -392,3 +392,82 @@ def test_fp8_random_shapes_and_ragged():
         if _run_fp8(c, rule=int(rng.integers(0, 3)), seed=it, integer=bool(it % 2)) is not None:
             done += 1
     assert done >= 5
+
+
+def test_fp8_wait_that_runs_out_reports_timeout():
+    """The same stalled epilogue with the converter warps running: every role,
+    converters included, stops at the wait limit and the status is TIMEOUT;
+    the next launch is correct."""
+    m = me()
+    c = _small(2, 512, 4, 2, 2, 256, 256)
+    cfgd = dict(c, payload="fp8")
+    cfg, bufs, o = _plan(cfgd, 1, 0)
+    assert o["status"] == 0
+    P = cfg.R * cfg.S * cfg.K
+    q, sc = _gen_fp8(P, cfg.H, 0, True)
+    home = _gen((cfg.E, cfg.H, cfg.Hp), 1, True)
+    w = _plain_weights(cfg, o, home)
+    y = torch.zeros((P, cfg.Hp), dtype=torch.bfloat16, device="cuda")
+    m.set_wait_limit_ns(20_000_000)
+    m.debug_set_barrier_extra(1)
+    try:
+        m.expert_gemm(cfg, bufs, torch.from_numpy(q).cuda(), w, y,
+                      recv_scale=torch.from_numpy(sc).cuda())
+        torch.cuda.synchronize()
+        assert m.plan_status(bufs)[0] == m.STATUS_TIMEOUT
+    finally:
+        m.debug_set_barrier_extra(0)
+        m.set_wait_limit_ns(1_000_000_000)
+    assert _run_fp8(c, rule=1, seed=0, integer=True) is not None
+
+
+def test_fp8_full_size_sampled():
+    """The fp8 workload at full size (R16 S16384 E128 K8 H4096, B8, H'=1536):
+    seeded e4m3 codes and scales drawn on the device, weights in VMM views
+    filled by the prefetch; sampled rows (every group's first and last rows,
+    tile edges, random rows of ten experts) against the dequantisation and
+    GEMM of the oracle."""
+    m = me()
+    cfgd = wl.WORKLOADS["fp8"]
+    cfg, bufs, o = _plan(cfgd, 0, 0)
+    assert o["status"] == 0
+    R, E, B, H, Hp = cfg.R, cfg.E, cfg.B, cfg.H, cfg.Hp
+    C = cfg.S * cfg.K
+    P = R * C
+    g = torch.Generator(device="cuda")
+    g.manual_seed(77)
+    q = torch.empty((P, H), dtype=torch.uint8, device="cuda")
+    for i in range(0, P, 1 << 18):
+        sl = q[i:i + (1 << 18)]
+        sl.copy_(torch.randint(0, 256, sl.shape, generator=g, device="cuda", dtype=torch.int32))
+        sl[(sl & 0x7F) == 0x7F] = 0x3C  # no NaN codes
+    sc = torch.exp2(torch.rand((P, H // 128), generator=g, device="cuda") * 4 - 8)
+    views = m.WeightViews(cfg, elem_bytes=2)
+    try:
+        v0 = m.weight_view_tensor(views, 0, cfg, torch.bfloat16)
+        v0[:E] = _gen((E, H, Hp), 4, False, scale=H ** -0.5)
+        m.prefetch(cfg, bufs, views.ptrs, 2)
+        y = torch.zeros((P, Hp), dtype=torch.bfloat16, device="cuda")
+        m.expert_gemm(cfg, bufs, q, views.ptrs[0], y, recv_scale=sc)
+        torch.cuda.synchronize()
+        assert m.plan_status(bufs)[0] == m.STATUS_OK
+        rows = _sample_rows(o, cfg, 64, seed=3)
+        ranks, groups = oracle.row_groups(E, B, C, o["cu_seqlens"], rows)
+        ex = _experts_of(cfg, o, ranks, groups)
+        chosen = np.unique(ex[groups >= E])[:5]
+        rest = np.setdiff1d(np.unique(ex), chosen)
+        chosen = np.concatenate([chosen, np.random.default_rng(4).choice(rest, 5, replace=False)])
+        rows = rows[np.isin(ex, chosen)]
+        assert len(rows) >= 40
+        rows_d = torch.from_numpy(rows).cuda()
+        q_rows = q[rows_d].cpu().numpy()
+        s_rows = sc[rows_d].cpu().numpy()
+        ranks, groups = oracle.row_groups(E, B, C, o["cu_seqlens"], rows)
+        experts = _experts_of(cfg, o, ranks, groups)
+        uniq, mat = np.unique(experts, return_inverse=True)
+        ref = oracle.expert_gemm_rows(oracle.dequant_rows(q_rows, s_rows), mat.astype(np.int32),
+                                      bits16(v0[torch.from_numpy(uniq).cuda()]))
+        _check(bits16(y[rows_d]), ref, H, False)
+        del v0
+    finally:
+        views.close()
