@@ -85,6 +85,16 @@ def test_backward_small_full(rule):
         _check_tokens(r, np.arange(cfgd["R"] * cfgd["S"]))
 
 
+@pytest.mark.parametrize("K,H", [(8, 256), (12, 512), (32, 64)])
+def test_backward_many_picks(K, H):
+    """Both sides of the K = 8 switch in the backward kernels, every token."""
+    cfgd = dict(name="bwd-k", R=2, S=40, E=32, K=K, B=16, H=H, Hp=0, routing="zipf",
+                alpha=0.5, expert="identity", payload="bf16")
+    r = _setup(cfgd, seed=1, rule=1)
+    assert r["o"]["status"] == 0
+    _check_tokens(r, np.arange(cfgd["R"] * cfgd["S"]))
+
+
 def test_backward_tiny_and_uniform_full():
     for name in ("tiny", "uniform"):
         cfgd = wl.WORKLOADS[name]

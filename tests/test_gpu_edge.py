@@ -47,6 +47,22 @@ def test_degenerate_and_ragged(shape):
             _full_check(cfgd, idx, w, seed=seed, rule=rule)
 
 
+@pytest.mark.parametrize("shape", [
+    (2, 48, 16, 8, 8, 256),     # K = 8: the all-K-first combine with every pick slot used
+    (2, 40, 16, 12, 8, 512),    # K = 12: the double-buffered combine and backward kernels
+    (4, 16, 32, 32, 16, 64),    # K = 32 = the largest K, every token picks every expert
+])
+def test_many_picks_per_token(shape):
+    """Above K = 8, combine and both backward kernels switch to the forms that
+    keep two picks in flight; both sides of that switch, bit-exact."""
+    R, S, E, K, B, H = shape
+    cfgd = _cfg(R, S, E, K, B, H, alpha=0.5)
+    for seed in range(2):
+        idx, w = wl.routing(cfgd, seed=seed)
+        for rule in (0, 2):
+            _full_check(cfgd, idx, w, seed=seed, rule=rule, expert="scale")
+
+
 def test_largest_E_and_R():
     cfgd = _cfg(128, 16, 1024, 8, 16, 64, alpha=1.2)
     idx, w = wl.routing(cfgd, seed=0)
