@@ -11,12 +11,18 @@
 // for sm_100a:
 //
 //  - one persistent CTA per SM: warp 0 issues TMA loads, one thread of warp 1
-//    issues tcgen05.mma, warps 2-5 drain the accumulator (192 threads); for
-//    the fp8 payload CW more warps widen the e4m3 rows to bf16 in shared
-//    memory (a = bf16(float(q) * scale)) between the TMA and the MMA;
-//  - tile 128 rows x BN columns (BN = 256 when H' allows, else 128), k-block
-//    64: A = 128 x 64 bf16 rows of the dispatched block (K-major), B = 64 x BN
-//    of the weight row (H' contiguous, MN-major), both 128-byte swizzled;
+//    issues tcgen05.mma, warps 2-5 drain the accumulator (192 threads);
+//  - bf16 payload: tile 128 rows x BN columns (BN = 256 when H' allows, else
+//    128), k-block 64: A = 128 x 64 bf16 rows of the dispatched block
+//    (K-major), B = 64 x BN of the weight row (H' contiguous, MN-major), both
+//    128-byte swizzled in shared memory;
+//  - fp8 payload: A never exists in bf16 outside the SM.  Warp 6 streams the
+//    e4m3 tiles into a ring of 8 slots, 8 converter warps widen them
+//    (a = bf16(float(q) * scale)) straight into tensor memory with
+//    tcgen05.st, and the MMA reads A from there; shared memory then holds
+//    only B.  Tiles are 128 x 192, so two accumulators (384 columns) and 4 A
+//    stages (32 columns each) fill the 512 columns; the last n-tile may be
+//    partial;
 //  - the fp32 accumulator lives in tensor memory, two buffers of BN columns,
 //    so the epilogue of one tile overlaps the main loop of the next;
 //  - the epilogue reads 32 lanes x 32 columns per tcgen05.ld, rounds once to
@@ -32,7 +38,7 @@
 //
 // Every wait is bounded by the library's wait limit (globaltimer).  A wait
 // that runs out raises a CTA-wide abort flag; each role then stops, the TMA
-// warp waits (bounded) for the loads it still has in flight, the MMA thread
+// warps wait (bounded) for the loads they still have in flight, the MMA thread
 // waits (bounded) for its issued MMAs to finish, TMEM is released, and the
 // plan's status becomes MOONEP_STATUS_TIMEOUT.
 #include <cuda.h>
@@ -48,9 +54,9 @@ constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int A_BYTES = BM * BK * 2;   // 16 KiB of bf16 A per stage
 constexpr int A8_BYTES = BM * BK;      // 8 KiB of e4m3 A per k-block (fp8 payload)
-// fp8 payload: CW extra warps widen A to bf16
+// fp8 payload: one more warp loads the e4m3 tiles and CW warps widen them
 template <bool FP8A, int CW>
-__host__ __device__ constexpr int threads_for() { return FP8A ? (6 + CW) * 32 : 6 * 32; }
+__host__ __device__ constexpr int threads_for() { return FP8A ? (7 + CW) * 32 : 6 * 32; }
 // dynamic shared memory a CTA may ask for: the 227 KiB opt-in limit less
 // room for the kernel's static shared variables
 constexpr int SMEM_LIMIT = 227 * 1024 - 256;
@@ -139,6 +145,51 @@ __device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
+// The same MMA with A read from tensor memory: `tmem_a` addresses lane 0 of
+// the 8 columns that hold the 128 x 16 bf16 A block (row i in lane i, two
+// elements per 32-bit column, the lower k in the low half).
+__device__ __forceinline__ void mma_bf16_tmem_a(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc,
+                                                uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p; }" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+// Store NW 32-bit words per lane into NW consecutive tensor-memory columns of
+// the warp's 32 lanes, and wait until the stores are done.
+template <int NW>
+__device__ __forceinline__ void tmem_store(uint32_t taddr, const uint32_t* v) {
+    static_assert(NW == 8 || NW == 16 || NW == 32, "8, 16 or 32 columns");
+    if constexpr (NW == 8) {
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(
+                         taddr),
+                     "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+                     "r"(v[7])
+                     : "memory");
+    } else if constexpr (NW == 16) {
+        asm volatile(
+            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+            "%13,%14,%15,%16};" ::"r"(taddr),
+            "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+            "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+            "r"(v[15])
+            : "memory");
+    } else {
+        asm volatile(
+            "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+            "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(
+                taddr),
+            "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+            "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+            "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+            "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+            "r"(v[29]), "r"(v[30]), "r"(v[31])
+            : "memory");
+    }
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 // Arrive on `bar` once every tcgen05 operation this thread issued is done.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
     asm volatile(
@@ -191,11 +242,19 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
                        const __grid_constant__ CUtensorMap tmW, GemmArgs p) {
     constexpr int THREADS = threads_for<FP8A, CW>();
     constexpr int B_BYTES = BK * BN * 2;
-    // a stage of the MMA ring: bf16 A (SW128, K-major) | B.  The fp8 payload
-    // lands in its own ring of A8_SLOTS e4m3 tiles after the stages.
-    constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    // a stage of the MMA ring: bf16 A (SW128, K-major) | B.  fp8 payload: A
+    // lives in tensor memory, so a stage holds only B, and the e4m3 tiles
+    // land in their own ring of A8_SLOTS after the stages.
+    constexpr int STAGE_A = FP8A ? 0 : A_BYTES;
+    constexpr int STAGE_BYTES = STAGE_A + B_BYTES;
     constexpr int A8S = FP8A ? A8_SLOTS : 0;
-    constexpr int TMEM_COLS = 2 * BN;
+    // two accumulators of BN columns; fp8 payload: then A stage s at columns
+    // ACOL + 32 s (128 rows x 64 bf16, two elements per column)
+    constexpr int ACOL = 2 * BN;
+    constexpr int TMEM_COLS = FP8A ? 512 : 2 * BN;
+    static_assert(!FP8A || (ACOL + 32 * STAGES <= 512 && CW % 4 == 0 && CW <= 16),
+                  "fp8 payload: two accumulators and the A stages in 512 columns, whole "
+                  "converter warps per lane quarter");
     // k-block of A: 128 rows x 128 B; one k-step (16 elements) = 32 B along a row.
     // k-block of B: BN/64 column chunks of 64 k-rows x 128 B (8 KiB each); one
     // k-step = 16 k-rows = 2 KiB; the next 64-column chunk is 8 KiB further.
@@ -213,7 +272,8 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
     uint64_t* never = drain + 1;
     uint32_t* tmem_slot = (uint32_t*)(never + 1);
     int* wsum = (int*)(tmem_slot + 2);  // [THREADS / 32]
-    int* pre = wsum + 16;               // [npairs + 1] m-tile prefix
+    int* pre = wsum + 32;               // [npairs + 1] m-tile prefix
+    static_assert(THREADS / 32 <= 32, "one per-warp sum slot per warp");
     __shared__ volatile int abort_flag;
     __shared__ int plan_status;
 
@@ -226,7 +286,7 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
     const int G = p.E + p.B;      // groups per rank
     const int per = p.Er + p.B;   // groups a plan can fill per rank
     const int npairs = p.R * per;
-    const int ntn = p.Hp / BN;
+    const int ntn = (p.Hp + BN - 1) / BN;  // the last n-tile may be partial
     const int kblocks = p.H / BK;
 
     if (tid == 0) {
@@ -323,6 +383,10 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
                 pair_rg(pair, r, g);
                 const int row0 = r * p.C + (g ? __ldg(p.cu + r * G + g - 1) : 0) + mt * BM;
                 const int wrow0 = (r * G + g) * p.H;
+                // 64-column boxes of B inside H' (all of them unless the
+                // last n-tile is partial; the rest of the stage is not read
+                // into any stored column)
+                const int nbox = min(BN / 64, (p.Hp - nt * BN) / 64);
                 bool ok = true;
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait(&empty[s], ph ^ 1, p.wait_ns, &abort_flag)) {
@@ -330,27 +394,18 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
                         break;
                     }
                     uint8_t* a = smem + s * STAGE_BYTES;
-                    uint8_t* b = a + A_BYTES;
-                    if constexpr (FP8A) {
-                        // the e4m3 tile goes to its own ring; the converters
-                        // widen it into this stage's A once it lands
-                        const int j8 = (int)(issued % A8S);
-                        const uint32_t p8 = (uint32_t)((issued / A8S) & 1);
-                        if (!mbar_wait(&a8empty[j8], p8 ^ 1, p.wait_ns, &abort_flag)) {
-                            ok = false;
-                            break;
-                        }
-                        mbar_expect_tx(&a8full[j8], A8_BYTES);
-                        tma_load_2d(a8ring + j8 * A8_BYTES, &tmX, &a8full[j8], kb * BK, row0);
-                        mbar_expect_tx(&full[s], B_BYTES);
+                    uint8_t* b = a + STAGE_A;
+                    if constexpr (FP8A) {  // A comes from the e4m3 producer and the converters
+                        mbar_expect_tx(&full[s], nbox * 8192);
                     } else {
-                        mbar_expect_tx(&full[s], A_BYTES + B_BYTES);
+                        mbar_expect_tx(&full[s], A_BYTES + nbox * 8192);
                         tma_load_2d(a, &tmX, &full[s], kb * BK, row0);
                     }
 #pragma unroll
                     for (int j = 0; j < BN / 64; ++j)
-                        tma_load_2d(b + j * 8192, &tmW, &full[s], nt * BN + 64 * j,
-                                    wrow0 + kb * BK);
+                        if (j < nbox)
+                            tma_load_2d(b + j * 8192, &tmW, &full[s], nt * BN + 64 * j,
+                                        wrow0 + kb * BK);
                     ++issued;
                     if (++s == STAGES) {
                         s = 0;
@@ -364,9 +419,6 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
                 // wait for the last STAGES of them to land before leaving
                 for (long long n = issued > STAGES ? issued - STAGES : 0; n < issued; ++n)
                     mbar_drain(&full[n % STAGES], (uint32_t)((n / STAGES) & 1), p.wait_ns);
-                if constexpr (FP8A)  // and the last e4m3 tiles
-                    for (long long n = issued > A8S ? issued - A8S : 0; n < issued; ++n)
-                        mbar_drain(&a8full[n % A8S], (uint32_t)((n / A8S) & 1), p.wait_ns);
             }
         }
     } else if (warp == 1) {
@@ -396,11 +448,17 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
                     }
                     asm volatile("tcgen05.fence::after_thread_sync;");
                     const uint32_t a = smem_u32(smem + s * STAGE_BYTES);
-                    const uint32_t b = a + A_BYTES;
+                    const uint32_t b = a + STAGE_A;
 #pragma unroll
-                    for (int ks = 0; ks < BK / 16; ++ks)
-                        mma_bf16(d, sdesc(a + ks * 32, 16, 1024), sdesc(b + ks * 2048, 8192, 1024),
-                                 idesc, (kb | ks) ? 1u : 0u);
+                    for (int ks = 0; ks < BK / 16; ++ks) {
+                        if constexpr (FP8A)
+                            mma_bf16_tmem_a(d, tmem + ACOL + s * 32 + ks * 8,
+                                            sdesc(b + ks * 2048, 8192, 1024), idesc,
+                                            (kb | ks) ? 1u : 0u);
+                        else
+                            mma_bf16(d, sdesc(a + ks * 32, 16, 1024),
+                                     sdesc(b + ks * 2048, 8192, 1024), idesc, (kb | ks) ? 1u : 0u);
+                    }
                     any = true;
                     mma_commit(&empty[s]);
                     if (++s == STAGES) {
@@ -439,6 +497,7 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
             const uint32_t tbase = tmem + acc * BN + ((uint32_t)(q * 32) << 16);
 #pragma unroll 1
             for (int c0 = 0; c0 < BN; c0 += 32) {
+                if (nt * BN + c0 >= p.Hp) break;  // partial last n-tile (warp-uniform)
                 uint32_t v[32];
                 asm volatile(
                     "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,"
@@ -473,65 +532,111 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
             }
         }
     } else if constexpr (FP8A) {
-        // converters: widen each e4m3 tile (row-major, 64 B a row) into the
-        // stage's bf16 A, in the 128-byte-swizzled K-major layout the MMA reads:
-        // a = bf16(float(q) * scale), one binary32 product, round to nearest
-        // even.  A warp reads 32 consecutive 16-byte chunks (8 rows) and
-        // writes each as two 16-byte bf16 chunks at their swizzled places.
-        const int ct = tid - 6 * 32;  // 0 .. CW*32 - 1
-        const int nsc = p.H / 128;    // scales per row
-        const long long nrows = (long long)p.R * p.C;
-        int s = 0;
-        long long n = 0;  // k-blocks converted: tile n % A8S of the e4m3 ring
-        for (int tile = blockIdx.x; tile < total && !abort_flag; tile += gridDim.x) {
-            int pair, mt, nt, r, g;
-            locate(tile, pair, mt, nt);
-            pair_rg(pair, r, g);
-            const long long row0 =
-                (long long)r * p.C + (g ? __ldg(p.cu + r * G + g - 1) : 0) + mt * BM;
-            bool ok = true;
-            for (int kb = 0; kb < kblocks; ++kb) {
-                // the tile landed; the producer loaded it only after this
-                // stage's previous MMAs finished, so the stage's A is free
-                const int j8 = (int)(n % A8S);
-                if (!mbar_wait(&a8full[j8], (uint32_t)((n / A8S) & 1), p.wait_ns, &abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                uint8_t* a16 = smem + s * STAGE_BYTES;
-                const uint8_t* a8 = a8ring + j8 * A8_BYTES;
-#pragma unroll
-                for (int j = 0; j < (BM * BK / 16) / (CW * 32); ++j) {
-                    const int chunk = j * CW * 32 + ct;
-                    const int row = chunk >> 2, cq = chunk & 3;
-                    const uint4 v = *reinterpret_cast<const uint4*>(a8 + chunk * 16);
-                    const long long grow = row0 + row;
-                    const float sc = grow < nrows ? __ldg(p.scale + grow * nsc + (kb >> 1)) : 0.0f;
-                    uint32_t o[8];
-                    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        o[2 * q] = widen_e4m3x2(w4[q] & 0xffffu, sc);
-                        o[2 * q + 1] = widen_e4m3x2(w4[q] >> 16, sc);
+        if (warp == 6) {
+            if (lane == 0) {  // e4m3 producer: runs up to A8S k-blocks ahead of the converters
+                long long issued = 0;
+                for (int tile = blockIdx.x; tile < total && !abort_flag; tile += gridDim.x) {
+                    int pair, mt, nt, r, g;
+                    locate(tile, pair, mt, nt);
+                    pair_rg(pair, r, g);
+                    const int row0 = r * p.C + (g ? __ldg(p.cu + r * G + g - 1) : 0) + mt * BM;
+                    bool ok = true;
+                    for (int kb = 0; kb < kblocks; ++kb) {
+                        const int j8 = (int)(issued % A8S);
+                        const uint32_t p8 = (uint32_t)((issued / A8S) & 1);
+                        if (!mbar_wait(&a8empty[j8], p8 ^ 1, p.wait_ns, &abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_expect_tx(&a8full[j8], A8_BYTES);
+                        tma_load_2d(a8ring + j8 * A8_BYTES, &tmX, &a8full[j8], kb * BK, row0);
+                        ++issued;
                     }
-                    const int sw = row & 7;
-                    uint8_t* dst = a16 + row * 128;
-                    *reinterpret_cast<uint4*>(dst + (((2 * cq) ^ sw) << 4)) =
-                        make_uint4(o[0], o[1], o[2], o[3]);
-                    *reinterpret_cast<uint4*>(dst + (((2 * cq + 1) ^ sw) << 4)) =
-                        make_uint4(o[4], o[5], o[6], o[7]);
+                    if (!ok) break;
                 }
-                // generic-proxy stores, read next by the tensor cores
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&conv[s]);
-                    mbar_arrive(&a8empty[j8]);
-                }
-                ++n;
-                if (++s == STAGES) s = 0;
+                if (abort_flag)  // wait for the last e4m3 tiles to land before leaving
+                    for (long long n = issued > A8S ? issued - A8S : 0; n < issued; ++n)
+                        mbar_drain(&a8full[n % A8S], (uint32_t)((n / A8S) & 1), p.wait_ns);
             }
-            if (!ok) break;
+        } else {
+            // converters, A in tensor memory: a thread owns one row of the tile
+            // (TMEM lane q*32 + lane, q = warp % 4, the lanes this warp may
+            // address) and CPT of its 64 codes per k-block.  It reads them from
+            // the e4m3 tile (64-byte swizzle: chunk c of row i sits at chunk
+            // c ^ ((i >> 1) & 3), so the 8 rows of a shared-memory phase hit 8
+            // distinct bank groups), widens them to bf16 = bf16(float(q) * scale)
+            // and stores them into the stage's A columns with tcgen05.st.
+            constexpr int PER_Q = CW / 4;      // converter warps per lane quarter
+            constexpr int CPT = 64 / PER_Q;    // codes per thread and k-block
+            constexpr int NCH = CPT / 16;      // 16-byte chunks per thread
+            constexpr int NW = CPT / 2;        // bf16x2 words = TMEM columns
+            const int q = warp & 3;
+            const int h = (warp - 7) >> 2;     // which CPT codes of the row
+            const int row = q * 32 + lane;
+            const int xr = (row >> 1) & 3;
+            const uint32_t tlane = tmem + ((uint32_t)(q * 32) << 16) + ACOL + h * NW;
+            const int nsc = p.H / 128;  // scales per row; one k-block uses scale kb / 2
+            const long long nrows = (long long)p.R * p.C;
+            int s = 0;
+            long long n = 0;  // k-blocks converted: tile n % A8S of the e4m3 ring
+            for (int tile = blockIdx.x; tile < total && !abort_flag; tile += gridDim.x) {
+                int pair, mt, nt, r, g;
+                locate(tile, pair, mt, nt);
+                pair_rg(pair, r, g);
+                const long long grow =
+                    (long long)r * p.C + (g ? __ldg(p.cu + r * G + g - 1) : 0) + mt * BM + row;
+                const bool live = grow < nrows;  // rows past the block are zero-filled
+                const float* srow = p.scale + (live ? grow * nsc : 0);
+                // the scale of the next 128 columns is loaded one group ahead
+                float sc = live ? __ldg(srow) : 0.0f;
+                float sc_next = live && nsc > 1 ? __ldg(srow + 1) : 0.0f;
+                bool ok = true;
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (kb > 0 && (kb & 1) == 0) {
+                        sc = sc_next;
+                        const int gi = (kb >> 1) + 1;
+                        sc_next = live && gi < nsc ? __ldg(srow + gi) : 0.0f;
+                    }
+                    // the e4m3 tile landed
+                    const int j8 = (int)(n % A8S);
+                    if (!mbar_wait(&a8full[j8], (uint32_t)((n / A8S) & 1), p.wait_ns, &abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint8_t* a8 = a8ring + j8 * A8_BYTES + row * 64;
+                    uint32_t o[NW];
+#pragma unroll
+                    for (int i = 0; i < NCH; ++i) {
+                        const int c = h * NCH + i;
+                        const uint4 v = *reinterpret_cast<const uint4*>(a8 + ((c ^ xr) << 4));
+                        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            o[8 * i + 2 * k] = widen_e4m3x2(w4[k] & 0xffffu, sc);
+                            o[8 * i + 2 * k + 1] = widen_e4m3x2(w4[k] >> 16, sc);
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&a8empty[j8]);  // the e4m3 tile is read
+                    // widened in registers first; now wait until the MMAs that
+                    // read this stage's A columns last (k-block n - STAGES) are
+                    // done, and order their reads before the stores
+                    if (!mbar_wait(&empty[s], (uint32_t)(((n / STAGES) & 1) ^ 1), p.wait_ns,
+                                   &abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    asm volatile("tcgen05.fence::after_thread_sync;");
+                    tmem_store<NW>(tlane + s * 32, o);
+                    // the tensor-memory stores complete before the MMA reads them
+                    asm volatile("tcgen05.fence::before_thread_sync;");
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&conv[s]);
+                    ++n;
+                    if (++s == STAGES) s = 0;
+                }
+                if (!ok) break;
+            }
         }
     }
     asm volatile("tcgen05.fence::before_thread_sync;");
@@ -578,8 +683,9 @@ bool encode_2d(CUtensorMap* m, const void* base, CUtensorMapDataType type, uint6
 // slot, 2 + 2 accumulator, drain, never) + TMEM address + per-warp sums +
 // the m-tile prefix
 size_t smem_bytes(int bn, int stages, int npairs, bool fp8a, int a8_slots = 2) {
-    return 1024 + (size_t)stages * (A_BYTES + BK * bn * 2) + (fp8a ? a8_slots * A8_BYTES : 0) +
-           (size_t)(3 * stages + 2 * a8_slots + 6) * 8 + 8 + 16 * 4 + (size_t)(npairs + 1) * 4;
+    return 1024 + (size_t)stages * ((fp8a ? 0 : A_BYTES) + BK * bn * 2) +
+           (fp8a ? a8_slots * A8_BYTES : 0) +
+           (size_t)(3 * stages + 2 * a8_slots + 6) * 8 + 8 + 32 * 4 + (size_t)(npairs + 1) * 4;
 }
 
 template <int BN, int STAGES, bool FP8A, int CW = 8, int A8_SLOTS = 2>
@@ -608,9 +714,11 @@ cudaError_t launch_variant(const CUtensorMap& x, const CUtensorMap& w, const Gem
 
 int expert_gemm_npairs(const moonep_config& c) { return c.R * (c.E / c.R + c.B); }
 
+// the fp8 kernel's configuration, or the smallest bf16 one
 bool expert_gemm_fits(const moonep_config& c) {
-    return smem_bytes(128, 3, expert_gemm_npairs(c), c.payload == MOONEP_PAYLOAD_FP8) <=
-           (size_t)SMEM_LIMIT;
+    const int np = expert_gemm_npairs(c);
+    return (c.payload == MOONEP_PAYLOAD_FP8 ? smem_bytes(192, 4, np, true, 8)
+                                            : smem_bytes(128, 3, np, false)) <= (size_t)SMEM_LIMIT;
 }
 
 cudaError_t launch_expert_gemm(const moonep_config& c, const moonep_plan_t& p, const void* x,
@@ -622,10 +730,11 @@ cudaError_t launch_expert_gemm(const moonep_config& c, const moonep_plan_t& p, c
     }
     const bool fp8 = c.payload == MOONEP_PAYLOAD_FP8;
     const int C = c.S * c.K;
+    const int np = expert_gemm_npairs(c);
     CUtensorMap tx, tw;
     const bool ok_x =
         fp8 ? encode_2d(&tx, x, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)c.H, (uint64_t)c.R * C,
-                        BK, BM, CU_TENSOR_MAP_SWIZZLE_NONE)
+                        BK, BM, CU_TENSOR_MAP_SWIZZLE_64B)
             : encode_2d(&tx, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)c.H,
                         (uint64_t)c.R * C, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok_x || !encode_2d(&tw, w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)c.Hp,
@@ -642,22 +751,10 @@ cudaError_t launch_expert_gemm(const moonep_config& c, const moonep_plan_t& p, c
     a.scale = x_scale;
     a.wait_ns = current_wait_limit_ns();
     a.debug_stall = current_barrier_extra() != 0;
-    const int np = expert_gemm_npairs(c);
     const int grid = device_sm_count();
-    if (fp8) {
-        // 4 MMA stages and 4 e4m3 tiles when they fit (29.5 ms at the fp8
-        // workload, against 30.1-31.3 ms with 2 tiles or 3 stages)
-        if (c.Hp % 256 == 0 && smem_bytes(256, 4, np, true, 4) <= (size_t)SMEM_LIMIT)
-            return launch_variant<256, 4, true, 8, 4>(tx, tw, a, smem_bytes(256, 4, np, true, 4),
-                                                      grid, s);
-        if (c.Hp % 256 == 0 && smem_bytes(256, 4, np, true) <= (size_t)SMEM_LIMIT)
-            return launch_variant<256, 4, true>(tx, tw, a, smem_bytes(256, 4, np, true), grid, s);
-        if (c.Hp % 256 == 0 && smem_bytes(256, 3, np, true) <= (size_t)SMEM_LIMIT)
-            return launch_variant<256, 3, true>(tx, tw, a, smem_bytes(256, 3, np, true), grid, s);
-        if (smem_bytes(128, 5, np, true) <= (size_t)SMEM_LIMIT)
-            return launch_variant<128, 5, true>(tx, tw, a, smem_bytes(128, 5, np, true), grid, s);
-        return launch_variant<128, 3, true>(tx, tw, a, smem_bytes(128, 3, np, true), grid, s);
-    }
+    if (fp8)  // 128 x 192 tiles: two accumulators and 4 A stages fill the 512 TMEM columns
+        return launch_variant<192, 4, true, 8, 8>(tx, tw, a, smem_bytes(192, 4, np, true, 8), grid,
+                                                  s);
     if (c.Hp % 256 == 0) {
         if (smem_bytes(256, 4, np, false) <= (size_t)SMEM_LIMIT)
             return launch_variant<256, 4, false>(tx, tw, a, smem_bytes(256, 4, np, false), grid, s);

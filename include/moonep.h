@@ -278,9 +278,10 @@ int moonep_expert_standin(const moonep_config* cfg, const moonep_plan_t* plan, c
  * recv:    the dispatched rows [R*C, H], rank r's rows at r*C
  *          (moonep_dispatch output): bf16, or for the fp8 payload e4m3 codes
  *          with recv_scale fp32 [R*C, H/128] (NULL for bf16).  fp8 rows are
- *          widened in shared memory to a = bf16(float(q) * scale), one
- *          binary32 product, round to nearest even -- the same values the
- *          identity stand-in expert produces -- and then multiplied as bf16.
+ *          widened on the SM, into tensor memory, to a = bf16(float(q) *
+ *          scale), one binary32 product, round to nearest even -- the same
+ *          values the identity stand-in expert produces -- and then
+ *          multiplied as bf16; no bf16 copy of them is written to memory.
  * weights: bf16, R consecutive [E+B, H, Hp] views; view r starts at element
  *          r*(E+B)*H*Hp.  Row e < E of a view is home expert e, row E+j is
  *          the replica in rank r's slot j.  The views of
