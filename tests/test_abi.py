@@ -102,3 +102,71 @@ def test_workspace_checked_by_the_planner_only(m):
     assert rc == m.ERR_INVALID_ARG and b"workspace" in m.lib.moonep_last_error()
     rc = m.lib.moonep_dispatch(ctypes.byref(cfg), ctypes.byref(plan), None, None, None, None)
     assert rc == m.ERR_INVALID_ARG and b"x or recv is NULL" in m.lib.moonep_last_error()
+
+
+def _fake_plan(m, slot=True):
+    """A plan whose pointers are aligned non-NULL addresses; the calls below
+    never get past their argument checks, so nothing reads them."""
+    f = 16
+    return m.Plan(f, f, f if slot else None, f, f, f, f, f, None, 0)
+
+
+# (call, config overrides, arguments after (cfg, plan), expected message)
+# Every case fails a check before any launch.
+_F, _U = 16, 24  # aligned and 8-byte (not 16-byte) aligned fake addresses
+_BAD_CALLS = [
+    ("moonep_expert_gemm", dict(payload=1, H=128, Hp=128), (_F, None, _F, _F, None), "needs recv_scale"),
+    ("moonep_expert_gemm", dict(payload=1, H=128, Hp=128), (_F, _U, _F, _F, None), "recv_scale must be 16-byte"),
+    ("moonep_expert_gemm", dict(H=72, Hp=128), (_F, None, _F, _F, None), "multiple of 64"),
+    ("moonep_expert_gemm", dict(Hp=0), (_F, None, _F, _F, None), "positive multiple of 128"),
+    ("moonep_expert_gemm", dict(Hp=192), (_F, None, _F, _F, None), "positive multiple of 128"),
+    ("moonep_expert_gemm", dict(Hp=128), (None, None, _F, _F, None), "NULL"),
+    ("moonep_expert_gemm", dict(Hp=128), (_F, None, _U, _F, None), "16-byte aligned"),
+    ("moonep_expert_standin", {}, (_F, None, 7, _F, None), "unknown mode"),
+    ("moonep_expert_standin", dict(payload=1, H=128), (_F, None, 0, _F, None), "needs recv_scale"),
+    ("moonep_expert_standin", {}, (_F, None, 0, _U, None), "16-byte aligned"),
+    ("moonep_dispatch", {}, (_F, _F, _F, None), "takes no recv_scale"),
+    ("moonep_dispatch", dict(payload=1, H=128), (_F, _F, None, None), "needs recv_scale"),
+    ("moonep_dispatch", dict(payload=1, H=128), (_F, _F, _F + 2, None), "4-byte aligned"),
+    ("moonep_dispatch", {}, (_U, _F, None, None), "16-byte aligned"),
+    ("moonep_combine", {}, (_F, None, _F, None), "NULL"),
+    ("moonep_combine", {}, (_F, _F, _U, None), "16-byte aligned"),
+    ("moonep_combine_backward", {}, (_F, _F, _F, _F, None, None), "NULL argument"),
+    ("moonep_combine_backward", {}, (_F, _U, _F, _F, _F, None), "16-byte aligned"),
+    ("moonep_dispatch_backward", {}, (_F, None, None), "NULL"),
+    ("moonep_dispatch_backward", {}, (_U, _F, None), "16-byte aligned"),
+]
+
+
+@pytest.mark.parametrize("fn,over,args,msg", _BAD_CALLS)
+def test_calls_check_arguments_before_any_launch(m, fn, over, args, msg):
+    d = dict(R=2, S=8, E=4, K=2, B=2, H=64, Hp=0, payload=0, rule=0)
+    d.update(over)
+    cfg = m.Config(**d)
+    plan = _fake_plan(m)
+    rc = getattr(m.lib, fn)(ctypes.byref(cfg), ctypes.byref(plan), *args)
+    assert rc == m.ERR_INVALID_ARG
+    assert msg in m.lib.moonep_last_error().decode(), m.lib.moonep_last_error()
+
+
+def test_side_kernels_check_views_and_skip_without_slots(m):
+    """prefetch and grad-reduce reject a missing or misaligned rank view and
+    return OK without launching when the plan has no slots (B = 0)."""
+    vp = ctypes.c_void_p
+    views = (vp * 2)(16, 24)
+    cfg = m.Config(2, 8, 4, 2, 2, 64, 128, 0, 0)
+    plan = _fake_plan(m)
+    assert m.lib.moonep_prefetch(ctypes.byref(cfg), ctypes.byref(plan), views, 2, None) == m.ERR_INVALID_ARG
+    assert b"16-byte aligned" in m.lib.moonep_last_error()
+    assert m.lib.moonep_prefetch(ctypes.byref(cfg), ctypes.byref(plan), views, 3, None) == m.ERR_INVALID_ARG
+    assert b"elem_bytes" in m.lib.moonep_last_error()
+    assert m.lib.moonep_grad_reduce(ctypes.byref(cfg), ctypes.byref(plan), None, None) == m.ERR_INVALID_ARG
+    assert b"rank_grads is NULL" in m.lib.moonep_last_error()
+    cfg0 = m.Config(2, 8, 4, 2, 0, 64, 128, 0, 0)
+    plan0 = _fake_plan(m, slot=False)
+    ok_views = (vp * 2)(16, 32)
+    assert m.lib.moonep_prefetch(ctypes.byref(cfg0), ctypes.byref(plan0), ok_views, 2, None) == m.OK
+    assert m.lib.moonep_grad_reduce(ctypes.byref(cfg0), ctypes.byref(plan0), ok_views, None) == m.OK
+    # a plan with slots needs slot_expert
+    rc = m.lib.moonep_prefetch(ctypes.byref(cfg), ctypes.byref(_fake_plan(m, slot=False)), ok_views, 2, None)
+    assert rc == m.ERR_INVALID_ARG and b"slot_expert" in m.lib.moonep_last_error()
