@@ -6,6 +6,11 @@ The C ABI is declared in include/moonep.h; the names here match it:
 ``moonep_plan`` -> :func:`plan`, ``moonep_dispatch`` -> :func:`dispatch`, and
 so on.  Importing this module fails loudly if the library has not been built;
 there is no fallback.
+
+Tensors are passed to the library as raw device addresses.  As in the C ABI,
+each buffer must be a contiguous CUDA allocation of at least the byte count
+:func:`sizes` gives for it: the library checks NULL pointers, alignment and
+the configuration, but it cannot see a buffer's extent.
 """
 import ctypes
 import os
