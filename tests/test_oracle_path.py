@@ -205,3 +205,27 @@ def test_dispatch_backward_closed_form(oracle_mod):
     mbig = oracle_mod.bf16_from_f32(np.array([-(2.0 ** 24)], np.float32))[0]
     seq = np.array([[[big], [one], [mbig], [one]]], np.uint16)  # ((2^24 + 1) - 2^24) + 1 = 1
     assert oracle_mod.bf16_to_f32(oracle_mod.dispatch_backward_tokens(seq))[0, 0] == 1.0
+
+
+def test_combine_fp8_identity_closed_form(oracle_mod):
+    """fp8 payload, identity expert, through the whole oracle path: every row
+    of token t dequantises to the same a[t] = bf16(float(q) * s), so y =
+    bf16(sum_k w_k a[t]).  a[t] is rebuilt here from torch alone (its e4m3
+    cast of x * (448/amax), its decode, binary32 multiply, bf16 cast), so the
+    quantisation, the dequantisation and the combine are all pinned from
+    outside the oracle."""
+    cfg, idx, w, x, pl = _small(oracle_mod, "tiny", H=384)
+    T, K, H = idx.shape[0], cfg["K"], 384
+    y, y64 = oracle_mod.path_tokens(cfg, x, w, pl, np.arange(T), expert="identity",
+                                    payload="fp8")
+    xv = torch.from_numpy(oracle_mod.bf16_to_f32(x)).view(T, H // 128, 128)
+    amax = xv.abs().amax(dim=2, keepdim=True)
+    inv = torch.where(amax > 0, torch.tensor(448.0) / amax, torch.ones_like(amax))
+    sc = torch.where(amax > 0, amax / torch.tensor(448.0), torch.ones_like(amax))
+    q = (xv * inv).to(torch.float8_e4m3fn).to(torch.float32)
+    a = (q * sc).view(T, H).to(torch.bfloat16).to(torch.float64).numpy()
+    exact = w.astype(np.float64).sum(1)[:, None] * a
+    assert np.allclose(y64, exact, rtol=1e-15, atol=0)
+    yv = oracle_mod.bf16_to_f32(y).astype(np.float64)
+    bound = np.abs(exact) * (2.0 ** -8 + K * 2.0 ** -23) * 1.0001
+    assert np.all(np.abs(yv - exact) <= bound)
