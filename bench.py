@@ -2,7 +2,7 @@
 synthetic routing, through the libmoonep C ABI.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl moonep|reference]
-                    [--workload uniform] [--alpha A] [--rule 0|1] [--sweep FILE]
+                    [--workload hot] [--alpha A] [--rule 0|1|2] [--no-sweep] [--sweep FILE]
 
 Prints one JSON line (rank 0).  Timing: W untimed warm-up steps; then K steps,
 each preceded by an L2 flush (a 512 MiB memset, then a 256 MiB read so that the
@@ -165,40 +165,64 @@ def rank_seed(base, rank):
 
 
 # ---------------------------------------------------------------- oracle arm
-def oracle_step_estimate(cfgd, idx, w, x_bits, rule, n_tokens, rng_seed=0, parts=None):
-    """One oracle step: the full plan, then dispatch, the identity stand-in
-    expert and combine for n sampled tokens, each timed and extrapolated to
-    all T tokens.  Returns (seconds for a full step, plan seconds, sample
-    seconds); `parts`, if given, receives the extrapolated seconds per step."""
+def oracle_sample_step(cfgd, idx, w, x_rows, rule, tokens):
+    """One step of the oracle on a bounded sample of the workload: the full
+    plan over all P picks, then dispatch, the identity stand-in expert and
+    combine of the sampled tokens only.  x_rows [n, H] holds the sampled
+    tokens' hidden states (bf16 bits).  Returns the seconds of each part."""
     import numpy as np
 
     import oracle
     R, S, E, K, B = (cfgd[k] for k in ("R", "S", "E", "K", "B"))
-    T, C = R * S, S * K
+    C = S * K
     fp8 = cfgd.get("payload") == "fp8"
+    tokens = np.asarray(tokens, np.int64)
     t0 = time.perf_counter()
     pl = oracle.plan(R, S, E, K, B, idx, rule=rule)
     t1 = time.perf_counter()
-    tokens = np.random.default_rng(rng_seed).choice(T, size=min(n_tokens, T), replace=False)
+    if pl["status"] != 0:
+        raise SystemExit("oracle plan failed with status %d (rule %d)" % (pl["status"], rule))
+    # a source map into the compact x_rows (harness bookkeeping, not timed)
     rows = pl["dst_row"][tokens].reshape(-1).astype(np.int64)
-    if fp8:
-        q, sc = oracle.dispatch_rows_fp8(K, x_bits, pl["src_of_row"], rows)
-    else:
-        recv = oracle.dispatch_rows(K, x_bits, pl["src_of_row"], rows)
+    src_c = np.zeros(R * S * K, np.int32)
+    src_c[rows] = np.arange(rows.size, dtype=np.int32)
     t2 = time.perf_counter()
+    if fp8:
+        q, sc = oracle.dispatch_rows_fp8(K, x_rows, src_c, rows)
+    else:
+        recv = oracle.dispatch_rows(K, x_rows, src_c, rows)
+    t3 = time.perf_counter()
     if fp8:
         eo = oracle.expert_rows("identity", E, B, C, pl, rows, q=q, s=sc)
     else:
         eo = oracle.expert_rows("identity", E, B, C, pl, rows, recv_bits=recv)
-    t3 = time.perf_counter()
-    oracle.combine_tokens(np.asarray(w, np.float32)[tokens], eo.reshape(tokens.size, K, -1))
     t4 = time.perf_counter()
-    scale = T / len(tokens)
-    full = (t1 - t0) + (t4 - t1) * scale
-    if parts is not None:
-        parts.update(plan_ms=(t1 - t0) * 1e3, dispatch_ms=(t2 - t1) * scale * 1e3,
-                     expert_ms=(t3 - t2) * scale * 1e3, combine_ms=(t4 - t3) * scale * 1e3)
-    return full, t1 - t0, t4 - t1
+    oracle.combine_tokens(np.asarray(w, np.float32)[tokens], eo.reshape(tokens.size, K, -1))
+    t5 = time.perf_counter()
+    return dict(plan=t1 - t0, dispatch=t3 - t2, expert=t4 - t3, combine=t5 - t4,
+                tokens=int(tokens.size))
+
+
+def oracle_rates(cfgd, parts):
+    """Measured seconds of a sample step, and the whole-workload step the
+    sample stands for (the plan already covers every pick; the per-token
+    parts scale with T / sampled tokens)."""
+    T = cfgd["R"] * cfgd["S"]
+    per_tok = parts["dispatch"] + parts["expert"] + parts["combine"]
+    measured = parts["plan"] + per_tok
+    full = parts["plan"] + per_tok * T / parts["tokens"]
+    return measured, full
+
+
+def calibrate_tokens(cfgd, idx, w, x_pool_fn, rule, budget_s, rng):
+    """Sampled-token count whose oracle step takes about budget_s seconds."""
+    T = cfgd["R"] * cfgd["S"]
+    n0 = min(256, T)
+    toks = rng.choice(T, size=n0, replace=False)
+    p = oracle_sample_step(cfgd, idx, w, x_pool_fn(n0), rule, toks)
+    per_tok = (p["dispatch"] + p["expert"] + p["combine"]) / n0
+    n = int((budget_s - p["plan"]) / max(per_tok, 1e-9))
+    return max(n0, min(T, n))
 
 
 def host_cpu():
@@ -215,39 +239,62 @@ def host_cpu():
 
 
 def run_reference(args, cfgd):
-    """The CPU oracle as the reference arm (rank 0 only)."""
+    """The CPU oracle as the reference arm (rank 0 only).  Each step is the
+    oracle on a bounded sample of the workload (full plan, sampled tokens'
+    dispatch/expert/combine), sized to about 1.5 s; ms_per_step is the
+    measured time of those steps."""
     import numpy as np
 
     from dispatch_moonep_plan_b200 import workloads as wl
-    world, rank, _ = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0
+    rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     import oracle
     oracle.lib()
-    T, P = cfgd["R"] * cfgd["S"], cfgd["R"] * cfgd["S"] * cfgd["K"]
+    T, P, H = cfgd["R"] * cfgd["S"], cfgd["R"] * cfgd["S"] * cfgd["K"], cfgd["H"]
     idx, w = wl.routing(cfgd, seed=rank_seed(0, 0), alpha=args.alpha)
-    x_bits = wl.bf16_bits(wl.hidden(T, cfgd["H"], seed=0))
-    n_tok = 256
+    rng = np.random.default_rng(0)
+    pool = {}
+
+    def x_pool(n):
+        # hidden states for the sampled tokens (same N(0,1) bf16 law as the
+        # GPU arm's x; drawn for the sample only)
+        if pool.get("n", 0) < n:
+            pool["x"] = wl.bf16_bits(wl.hidden(n, H, seed=0))
+            pool["n"] = n
+        return pool["x"][:n]
+
+    n_tok = calibrate_tokens(cfgd, idx, w, x_pool, args.rule, 1.5, rng)
+    xs = x_pool(n_tok)
     for _ in range(args.warmup):
-        oracle_step_estimate(cfgd, idx, w, x_bits, args.rule, n_tok)
-    steps = []
-    parts = {}
+        oracle_sample_step(cfgd, idx, w, xs, args.rule, rng.choice(T, n_tok, replace=False))
+    measured, full, parts = [], [], None
     t0 = time.perf_counter()
-    for i in range(args.steps):
-        steps.append(oracle_step_estimate(cfgd, idx, w, x_bits, args.rule, n_tok, rng_seed=i,
-                                          parts=parts)[0])
+    for _ in range(args.steps):
+        parts = oracle_sample_step(cfgd, idx, w, xs, args.rule,
+                                   rng.choice(T, n_tok, replace=False))
+        m, f = oracle_rates(cfgd, parts)
+        measured.append(m)
+        full.append(f)
     wall = time.perf_counter() - t0
-    step_s = statistics.mean(steps)
-    value = P / step_s
+    step_s = statistics.mean(measured)
+    full_s = statistics.mean(full)
+    value = P / full_s
     sample = ("each step: the full oracle plan over all %d picks, then dispatch + identity "
-              "expert + combine of %d sampled tokens, time extrapolated to all %d tokens"
-              % (P, n_tok, T))
+              "expert + combine of %d of the %d tokens (a fresh random sample each step); "
+              "ms_per_step is the measured time of such a step; value = all %d picks / the "
+              "whole-workload step time that the sample stands for (plan time + per-token time "
+              "x %d tokens), given under 'extrapolated'" % (P, n_tok, T, P, T))
     line = dict(impl="reference", metric=METRIC, value=value, unit=UNIT, n_gpus=args.gpus,
                 steps=args.steps, warmup=args.warmup, ms_per_step=step_s * 1e3,
                 higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16",
                 data="synthetic", config=workload_config(cfgd, args),
                 cpu_baseline=dict(kind="oracle", value=value, unit=UNIT, cores=1, sample=sample,
-                                  last_step_parts=parts, **host_cpu()),
+                                  sampled_tokens=n_tok,
+                                  last_step_s={k: v for k, v in parts.items() if k != "tokens"},
+                                  **host_cpu()),
+                extrapolated=dict(ms_per_full_step=full_s * 1e3, picks_per_full_step=P,
+                                  how="plan seconds + sampled per-token seconds x T / n"),
                 e2e=dict(value=value, unit=UNIT, h2d_bytes_per_step=0, d2h_bytes_per_step=0),
                 wall_s=wall)
     print(json.dumps(line), flush=True)
@@ -410,7 +457,7 @@ def run_gpu(args, cfgd, emit=True):
         clocks=clocks, clocks_per_kernel_pass=clk.summary(),
     )
     if emit and not args.no_side:
-        out["backward"] = measure_backward(me, cfg, bufs, T, P, H, K, flush, world)
+        out["backward"] = measure_backward(me, cfg, bufs, T, P, H, K, flush, world, eo)
         out["side"] = measure_side(me, wl, flush, world)
         out["expert_gemm"] = measure_gemm(me, wl, flush, world, local=local)
         out["expert_gemm_fp8"] = measure_gemm_fp8(me, wl, flush, world, local=local)
@@ -550,12 +597,14 @@ def e2e_pipelined(me, cfg, bufs, x, idx, w, recv, scale, eo, fp8, args, world):
     return dict(ms=ms, serial_ms=serial, h2d=h2d, d2h=d2h)
 
 
-def measure_backward(me, cfg, bufs, T, P, H, K, flush, world, reps=10):
+def measure_backward(me, cfg, bufs, T, P, H, K, flush, world, eo, reps=10):
     """Backward of combine (d_expert_out = w * dy per row, d_w = <dy, row>) and
-    of dispatch (dx = sum of the token's K rows) on the bench's workload."""
+    of dispatch (dx = sum of the token's K rows) on the bench's workload.  eo
+    is the step's bf16 expert output [P, H] (the forward's combine input)."""
     import torch
-    dy = torch.randn((T, H), device="cuda").to(torch.bfloat16)
-    eo = torch.randn((P, H), device="cuda").to(torch.bfloat16)
+
+    from dispatch_moonep_plan_b200 import workloads as wl
+    dy = wl.hidden(T, H, seed=77, device="cuda")
     w = torch.rand((T, K), device="cuda")
     d_eo = torch.empty_like(eo)
     d_w = torch.empty((T, K), dtype=torch.float32, device="cuda")
@@ -583,17 +632,23 @@ def measure_backward(me, cfg, bufs, T, P, H, K, flush, world, reps=10):
                combine_backward_frac=cb / tc / 1e6 / peak,
                dispatch_backward_us=td * 1e3, dispatch_backward_GBps=db / td / 1e6,
                dispatch_backward_frac=db / td / 1e6 / peak)
-    del dy, eo, d_eo, dx
+    del dy, d_eo, dx
     torch.cuda.empty_cache()
     return out
 
 
-def measure_side(me, wl, flush, world, reps=10):
+def measure_side(me, wl, flush, world, reps=10, S=None, Hp=None):
     """Replica prefetch (bf16 weights) and replica grad-reduce (fp32 grads) at
-    the fp8 workload's sizes on VMM-aliased [E+B, H, H'] views."""
+    the fp8 workload's sizes on VMM-aliased [E+B, H, H'] views (S, if given,
+    shrinks only the routing that places the slots; Hp the weight rows)."""
     import numpy as np
     import torch
-    cfgd = wl.WORKLOADS["fp8"]
+    kw = {}
+    if S:
+        kw["S"] = S
+    if Hp:
+        kw["Hp"] = Hp
+    cfgd = wl.cfg_with("fp8", **kw)
     cfg = me.config_from(cfgd, 0)
     idx, _ = wl.routing(cfgd, seed=0)
     bufs = me.PlanBuffers(cfg)
@@ -821,21 +876,34 @@ def measure_gemm_fp8(me, wl, flush, world, reps=5, S=None, local=None, rule=0):
 
 
 def cpu_baseline(cfgd, idx, w, x_dev, rule, budget_s=12.0):
-    """The oracle, as it stands, on a bounded sample of the same workload."""
+    """The oracle, as it stands, on a bounded sample of the same workload:
+    the full plan plus the sampled tokens' dispatch / identity expert /
+    combine, sized to about budget_s of one host core, rated over the whole
+    workload (value = all picks / the step time the sample stands for)."""
+    import numpy as np
+    import torch
+
     from dispatch_moonep_plan_b200 import workloads as wl
-    x_bits = wl.bf16_bits(x_dev)
     T, P = cfgd["R"] * cfgd["S"], cfgd["R"] * cfgd["S"] * cfgd["K"]
-    n = 256
-    full, tp, ts = oracle_step_estimate(cfgd, idx, w, x_bits, rule, n)
-    # grow the sample to use about budget_s of CPU time
-    per_tok = ts / n
-    n2 = int(max(n, min(T, (budget_s - tp) / max(per_tok, 1e-9))))
-    parts = {}
-    full, tp, ts = oracle_step_estimate(cfgd, idx, w, x_bits, rule, n2, rng_seed=1, parts=parts)
+    rng = np.random.default_rng(1)
+
+    def x_rows(tokens):
+        return wl.bf16_bits(x_dev[torch.from_numpy(np.asarray(tokens, np.int64)).cuda()])
+
+    n0 = min(256, T)
+    t0 = rng.choice(T, n0, replace=False)
+    p0 = oracle_sample_step(cfgd, idx, w, x_rows(t0), rule, t0)
+    per_tok = (p0["dispatch"] + p0["expert"] + p0["combine"]) / n0
+    n = int(max(n0, min(T, (budget_s - p0["plan"]) / max(per_tok, 1e-9))))
+    toks = np.sort(rng.choice(T, n, replace=False))
+    parts = oracle_sample_step(cfgd, idx, w, x_rows(toks), rule, toks)
+    measured, full = oracle_rates(cfgd, parts)
     return dict(kind="oracle", value=P / full, unit=UNIT, cores=1,
                 sample="full oracle plan (%d picks, %.3f s) + dispatch/identity expert/combine "
-                       "of %d of %d tokens (%.2f s), extrapolated to the whole step"
-                       % (P, tp, n2, T, ts), ms_per_step=full * 1e3, **parts, **host_cpu())
+                       "of %d of %d tokens (%.2f s measured), rated over the whole step"
+                       % (P, parts["plan"], n, T, measured - parts["plan"]),
+                ms_per_full_step=full * 1e3, measured_s=measured,
+                parts_s={k: v for k, v in parts.items() if k != "tokens"}, **host_cpu())
 
 
 def main(argv=None):
@@ -844,20 +912,30 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="moonep", choices=["moonep", "reference"])
-    ap.add_argument("--workload", default="uniform")
+    ap.add_argument("--workload", default="hot",
+                    help="the step's workload (default: the largest single-GPU one, R32 S8192 "
+                         "E384 K8 H7168 with half of all picks on one expert)")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="leave out the skew sweep and the other workloads' points")
     ap.add_argument("--alpha", type=float, default=None)
     ap.add_argument("--S", type=int, default=None,
                     help="tokens per rank, overriding the workload's (for small profiling cases)")
     ap.add_argument("--rule", type=int, default=0)
     ap.add_argument("--Hp", type=int, default=None,
-                    help="with --gemm-only: the expert output width H' (default: the workload's, "
-                         "else 1536)")
+                    help="with --gemm-only or --side-only: the expert output width H' (default: "
+                         "the workload's, else 1536)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-side", action="store_true",
                     help="skip the replica prefetch / grad-reduce measurement")
     ap.add_argument("--gemm-only", action="store_true",
                     help="time only the grouped expert GEMM (--S shrinks it; --workload fp8 takes "
                          "the fp8 payload) and print its line")
+    ap.add_argument("--side-only", action="store_true",
+                    help="time only the replica prefetch and grad-reduce (fp8 workload's "
+                         "routing and weight sizes; --S shrinks the routing) and print their line")
+    ap.add_argument("--backward-only", action="store_true",
+                    help="time only the backward of combine and of dispatch on --workload "
+                         "(--S shrinks it) and print their line")
     ap.add_argument("--sweep", default=None,
                     help="also time every workload / skew and write JSON lines to this file")
     args = ap.parse_args(argv)
@@ -874,11 +952,49 @@ def main(argv=None):
     if args.gemm_only:
         run_gemm_only(args)
         return
+    if args.side_only or args.backward_only:
+        run_part_only(args, cfgd)
+        return
     out = run_gpu(args, cfgd)
+    if out is not None and int(os.environ.get("WORLD_SIZE", "1")) == 1 and not args.no_sweep:
+        out["sweep"] = skew_sweep(args)
+        out["other_workloads"] = other_workloads(args)
     if out is not None:
         print(json.dumps(out), flush=True)
     if args.sweep and out is not None:
         run_sweep(args)
+
+
+def run_part_only(args, cfgd):
+    """One side measurement on its own (the small ncu cases): the replica
+    prefetch and grad-reduce, or the two backward kernels."""
+    import torch
+
+    from dispatch_moonep_plan_b200 import moonep as me
+    from dispatch_moonep_plan_b200 import workloads as wl
+    flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    def flush():
+        flush_w.zero_()
+
+    if args.side_only:
+        print(json.dumps(dict(side=measure_side(me, wl, flush, 1, reps=args.steps, S=args.S,
+                                                Hp=args.Hp))), flush=True)
+        return
+    cfg = me.config_from(dict(cfgd, payload="bf16"), args.rule)
+    s = me.sizes(cfg)
+    T, P, H, K = s.tokens, s.picks, cfg.H, cfg.K
+    idx, _ = wl.routing(cfgd, seed=0, alpha=args.alpha)
+    bufs = me.PlanBuffers(cfg)
+    me.plan(cfg, torch.from_numpy(idx).cuda(), bufs)
+    torch.cuda.synchronize()
+    st = me.plan_status(bufs)
+    if st[0] != me.STATUS_OK:
+        raise SystemExit("plan failed with status %s (rule %d)" % (st, args.rule))
+    eo = wl.hidden(P, H, seed=3, device="cuda")
+    out = measure_backward(me, cfg, bufs, T, P, H, K, flush, 1, eo, reps=args.steps)
+    out["workload"] = cfgd["name"]
+    print(json.dumps(dict(backward=out)), flush=True)
 
 
 def run_gemm_only(args):
@@ -898,6 +1014,68 @@ def run_gemm_only(args):
     out = measure_gemm(me, wl, flush, 1, reps=args.steps, S=args.S, rule=args.rule, base=base,
                        Hp=args.Hp)
     print(json.dumps(dict(expert_gemm=out)), flush=True)
+
+
+def _point(out, **extra):
+    """The per-workload figures of one run_gpu() result."""
+    keys = ("value", "ms_per_step", "maxvio", "plan_us", "dispatch_us", "combine_us",
+            "dispatch_GBps", "combine_GBps", "dispatch_frac", "combine_frac", "tokens_per_s",
+            "dtype", "clocks")
+    d = {k: out[k] for k in keys}
+    d["workload"] = out["config"]["workload"]
+    d["rule"] = out["config"]["rule"]
+    d["routed_rows_per_s"] = d.pop("value")
+    d.update(extra)
+    return d
+
+
+def _sub_args(args, alpha, rule):
+    a = argparse.Namespace(**vars(args))
+    a.alpha, a.rule, a.no_cpu_baseline, a.no_side, a.no_e2e = alpha, rule, True, True, True
+    a.steps = min(args.steps, 50)
+    a.warm_l2 = False
+    return a
+
+
+def skew_sweep(args):
+    """Routed rows/s against maxvio: the Zipf workload (R8 S4096 E256 K8
+    H7168 B16) at alpha 0, 0.5, 1.0, 1.5.  Rule 0 where it plans; where it
+    needs more than B slots (it fails loudly, as the oracle does) the point
+    is taken under rule 1 and the rule-0 failure is recorded beside it."""
+    import torch
+    from dispatch_moonep_plan_b200 import workloads as wl
+    pts = []
+    for alpha in wl.WORKLOADS["zipf"]["alphas"]:
+        rule0 = None
+        for rule in (0, 1):
+            try:
+                out = run_gpu(_sub_args(args, alpha, rule), wl.WORKLOADS["zipf"], emit=False)
+                pts.append(_point(out, alpha=alpha, rule0_failure=rule0))
+                break
+            except SystemExit as e:
+                rule0 = str(e)
+            finally:
+                torch.cuda.empty_cache()
+        else:
+            pts.append(dict(alpha=alpha, failed=rule0))
+    return pts
+
+
+def other_workloads(args):
+    """The other configurations, one point each: near-uniform routing (R8
+    S4096 E64 K6 H2048), the fp8 payload (R16 S16384 E128 K8 H4096, Zipf
+    1.2) and the distinct-pick reading of the hot expert."""
+    import torch
+    from dispatch_moonep_plan_b200 import workloads as wl
+    pts = []
+    for name in ("uniform", "fp8", "hot_tokens"):
+        try:
+            out = run_gpu(_sub_args(args, None, 0), wl.WORKLOADS[name], emit=False)
+            pts.append(_point(out))
+        except SystemExit as e:
+            pts.append(dict(workload=name, failed=str(e)))
+        torch.cuda.empty_cache()
+    return pts
 
 
 def run_sweep(args):

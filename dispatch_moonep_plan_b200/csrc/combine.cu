@@ -54,7 +54,7 @@ __global__ void __launch_bounds__(THREADS) combine_kernel(const uint4* __restric
                                                          const float* __restrict__ w,
                                                          const int32_t* __restrict__ dst_row,
                                                          uint4* __restrict__ y,
-                                                         const int32_t* __restrict__ status, int T,
+                                                         int32_t* status, int T,
                                                          int K, int H8) {
     if (load_status(status) != MOONEP_STATUS_OK) return;
     const int lane = threadIdx.x & 31;
@@ -64,7 +64,10 @@ __global__ void __launch_bounds__(THREADS) combine_kernel(const uint4* __restric
         // the last tokens last, so those are the rows still held in L2
         const long long t = WEIGHTED ? T - 1 - i : i;
         int myrow = lane < K ? __ldg(dst_row + t * K + lane) : 0;
-        if ((unsigned)myrow >= (unsigned)(T * K)) myrow = 0;  // range guard
+        if ((unsigned)myrow >= (unsigned)(T * K)) {  // range guard: report, read row 0
+            report_internal(status);
+            myrow = 0;
+        }
         const float myw = (WEIGHTED && lane < K) ? __ldg(w + t * K + lane) : 1.0f;
         for (int c0 = 0; c0 < H8; c0 += 32 * U) {
             float acc[U][8];
@@ -125,8 +128,8 @@ __global__ void __launch_bounds__(THREADS) combine_kfirst_kernel(const uint4* __
                                                                 const float* __restrict__ w,
                                                                 const int32_t* __restrict__ dst_row,
                                                                 uint4* __restrict__ y,
-                                                                const int32_t* __restrict__ status,
-                                                                int T, int K, int H8) {
+                                                                int32_t* status, int T, int K,
+                                                                int H8) {
     if (load_status(status) != MOONEP_STATUS_OK) return;
     const int lane = threadIdx.x & 31;
     const long long nw = (long long)gridDim.x * WARPS;
@@ -135,7 +138,10 @@ __global__ void __launch_bounds__(THREADS) combine_kfirst_kernel(const uint4* __
         // the last tokens last, so those are the rows still held in L2
         const long long t = WEIGHTED ? T - 1 - i : i;
         int myrow = lane < K ? __ldg(dst_row + t * K + lane) : 0;
-        if ((unsigned)myrow >= (unsigned)(T * K)) myrow = 0;  // range guard
+        if ((unsigned)myrow >= (unsigned)(T * K)) {  // range guard: report, read row 0
+            report_internal(status);
+            myrow = 0;
+        }
         const float myw = (WEIGHTED && lane < K) ? __ldg(w + t * K + lane) : 1.0f;
         long long base[KMAX];
         float wk[KMAX];
@@ -193,15 +199,18 @@ __global__ void __launch_bounds__(THREADS, 2) combine_bwd_kernel(const uint4* __
                                                              const int32_t* __restrict__ dst_row,
                                                              uint4* __restrict__ d_eo,
                                                              float* __restrict__ d_w,
-                                                             const int32_t* __restrict__ status,
-                                                             int T, int K, int H8) {
+                                                             int32_t* status, int T, int K,
+                                                             int H8) {
     if (load_status(status) != MOONEP_STATUS_OK) return;
     const int lane = threadIdx.x & 31;
     const int P = T * K;
     const long long nw = (long long)gridDim.x * WARPS;
     for (long long t = (long long)blockIdx.x * WARPS + (threadIdx.x >> 5); t < T; t += nw) {
         int myrow = lane < K ? __ldg(dst_row + t * K + lane) : 0;
-        if ((unsigned)myrow >= (unsigned)P) myrow = 0;  // range guard
+        if ((unsigned)myrow >= (unsigned)P) {  // range guard: report, use row 0
+            report_internal(status);
+            myrow = 0;
+        }
         const float myw = lane < K ? __ldg(w + t * K + lane) : 0.0f;
         long long base[KMAX];
         float wk[KMAX];
@@ -273,15 +282,18 @@ __global__ void __launch_bounds__(THREADS) combine_bwd_seq_kernel(const uint4* _
                                                              const int32_t* __restrict__ dst_row,
                                                              uint4* __restrict__ d_eo,
                                                              float* __restrict__ d_w,
-                                                             const int32_t* __restrict__ status,
-                                                             int T, int K, int H8) {
+                                                             int32_t* status, int T, int K,
+                                                             int H8) {
     if (load_status(status) != MOONEP_STATUS_OK) return;
     const int lane = threadIdx.x & 31;
     const int P = T * K;
     const long long nw = (long long)gridDim.x * WARPS;
     for (long long t = (long long)blockIdx.x * WARPS + (threadIdx.x >> 5); t < T; t += nw) {
         int myrow = lane < K ? __ldg(dst_row + t * K + lane) : 0;
-        if ((unsigned)myrow >= (unsigned)P) myrow = 0;  // range guard
+        if ((unsigned)myrow >= (unsigned)P) {  // range guard: report, use row 0
+            report_internal(status);
+            myrow = 0;
+        }
         const float myw = lane < K ? __ldg(w + t * K + lane) : 0.0f;
         float part[KMAX];
 #pragma unroll

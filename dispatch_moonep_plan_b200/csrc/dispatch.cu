@@ -24,14 +24,15 @@ template <int U>
 __global__ void __launch_bounds__(THREADS) dispatch_bf16_kernel(const uint4* __restrict__ x,
                                                                uint4* __restrict__ recv,
                                                                const int32_t* __restrict__ dst_row,
-                                                               const int32_t* __restrict__ status,
-                                                               int T, int K, int H8) {
+                                                               int32_t* status, int T, int K,
+                                                               int H8) {
     const int P = T * K;
     if (load_status(status) != MOONEP_STATUS_OK) return;
     const int lane = threadIdx.x & 31;
     const long long nw = (long long)gridDim.x * WARPS;
     for (long long t = (long long)blockIdx.x * WARPS + (threadIdx.x >> 5); t < T; t += nw) {
         const int myrow = lane < K ? __ldg(dst_row + t * K + lane) : 0;
+        if (lane < K && (unsigned)myrow >= (unsigned)P) report_internal(status);
         const uint4* src = x + t * H8;
         for (int c0 = 0; c0 < H8; c0 += 32 * U) {
             uint4 v[U];
@@ -42,7 +43,7 @@ __global__ void __launch_bounds__(THREADS) dispatch_bf16_kernel(const uint4* __r
             }
             for (int k = 0; k < K; ++k) {
                 const int row = __shfl_sync(0xffffffffu, myrow, k);
-                if ((unsigned)row >= (unsigned)P) continue;  // range guard
+                if ((unsigned)row >= (unsigned)P) continue;  // range guard (reported above)
                 uint4* dst = recv + (long long)row * H8;
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
@@ -74,8 +75,8 @@ __global__ void __launch_bounds__(THREADS) dispatch_fp8_kernel(const uint4* __re
                                                               uint8_t* __restrict__ recv,
                                                               float* __restrict__ recv_scale,
                                                               const int32_t* __restrict__ dst_row,
-                                                              const int32_t* __restrict__ status,
-                                                              int T, int K, int H8) {
+                                                              int32_t* status, int T, int K,
+                                                              int H8) {
     if (load_status(status) != MOONEP_STATUS_OK) return;
     extern __shared__ float row_scales[];  // [WARPS][H8/16]
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -87,6 +88,7 @@ __global__ void __launch_bounds__(THREADS) dispatch_fp8_kernel(const uint4* __re
     const long long nw = (long long)gridDim.x * WARPS;
     for (long long t = (long long)blockIdx.x * WARPS + warp; t < T; t += nw) {
         const int myrow = lane < K ? __ldg(dst_row + t * K + lane) : 0;
+        if (lane < K && (unsigned)myrow >= (unsigned)P) report_internal(status);
         const uint4* src = x + t * H8;
         for (int m0 = 0; m0 < nunits; m0 += 32 * U) {
             uint4 q[U];
@@ -127,7 +129,7 @@ __global__ void __launch_bounds__(THREADS) dispatch_fp8_kernel(const uint4* __re
             }
             for (int k = 0; k < K; ++k) {
                 const long long row = __shfl_sync(0xffffffffu, myrow, k);
-                if ((unsigned long long)row >= (unsigned long long)P) continue;  // range guard
+                if ((unsigned long long)row >= (unsigned long long)P) continue;  // range guard (reported above)
                 uint8_t* dst = recv + row * H;
 #pragma unroll
                 for (int u = 0; u < U; ++u) {

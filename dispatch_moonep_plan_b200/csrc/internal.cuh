@@ -68,6 +68,15 @@ __device__ __forceinline__ int load_status(const int32_t* status)
     return __ldcg(status + ST_STATUS);
 }
 
+// A kernel's own range check found an index outside its buffers (a planner
+// bug, or a plan the caller overwrote): record MOONEP_STATUS_INTERNAL in the
+// status block, unless an earlier failure is already there.  The caller skips
+// or clamps the access, so nothing is read or written out of range.
+__device__ __forceinline__ void report_internal(int32_t* status)
+{
+    atomicMax(status + ST_STATUS, MOONEP_STATUS_INTERNAL);
+}
+
 // ---- launchers (one per kernel file) ---------------------------------------
 struct PlanLaunch {
     int R, S, E, K, B, rule;

@@ -14,9 +14,16 @@
 // workspace, for up to MOONEP_NOALLOC_MAX_E experts (4 MiB + 2 KiB).  Every
 // GPU that loads the library holds it until the process exits.
 //
-// Host code cannot use the array's name as a device address: the address is
-// looked up with cudaGetSymbolAddress once per device, with that device
-// current, on the first call made on that device, and cached.
+// Host code cannot use the array's name as a device address.  The address
+// belongs to the driver context the library's module is loaded in, so it is
+// looked up with cudaGetSymbolAddress, with the calling device current, on
+// every call made outside a stream capture, and cached per device together
+// with that context.  A call inside a capture may not look anything up; it
+// takes the cached address, which must belong to the current context (after
+// a device reset, or under another driver context, the array lives at a new
+// address and the cache is stale until a call outside capture refreshes it).
+#include <cuda.h>
+
 #include <mutex>
 
 #include "internal.cuh"
@@ -29,25 +36,59 @@ constexpr size_t kScratchWords =
 static __device__ __align__(256) int32_t g_plan_scratch[kScratchWords];
 
 constexpr int kMaxDevices = 64;
+struct CachedAddress {
+    CUcontext ctx;
+    void* addr;
+};
 std::mutex g_mu;
-void* g_scratch_addr[kMaxDevices] = {};
+CachedAddress g_scratch_addr[kMaxDevices] = {};
 
 const char* const kFn = "moonep_plan_noalloc";
 
-// Device address of the scratch array on the current device.
-cudaError_t scratch_address(void** out) {
+using PFN_CtxGetCurrent = CUresult (*)(CUcontext*);
+
+// The driver context current on this thread (nullptr if none or unknown).
+CUcontext current_context() {
+    static PFN_CtxGetCurrent fn = [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            f = nullptr;
+        return reinterpret_cast<PFN_CtxGetCurrent>(f);
+    }();
+    CUcontext c = nullptr;
+    if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+    return c;
+}
+
+// Device address of the scratch array in the current device's context.
+cudaError_t scratch_address(cudaStream_t stream, void** out, const char** why) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    e = cudaStreamIsCapturing(stream, &cap);
+    if (e != cudaSuccess) return e;
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_addr[dev]) {
+    if (cap == cudaStreamCaptureStatusNone) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_plan_scratch);
         if (e != cudaSuccess) return e;
-        g_scratch_addr[dev] = p;
+        g_scratch_addr[dev].ctx = current_context();
+        g_scratch_addr[dev].addr = p;
+        *out = p;
+        return cudaSuccess;
     }
-    *out = g_scratch_addr[dev];
+    const CachedAddress& c = g_scratch_addr[dev];
+    if (!c.addr || c.ctx == nullptr || c.ctx != current_context()) {
+        *why = "inside a stream capture, but no call outside capture has looked up the scratch "
+               "array's address in this device's current context yet (first call, device reset "
+               "or another driver context): call it once before capturing";
+        return cudaErrorStreamCaptureUnsupported;
+    }
+    *out = c.addr;
     return cudaSuccess;
 }
 
@@ -70,9 +111,11 @@ extern "C" int moonep_plan_noalloc(const moonep_config* c, const int32_t* topk_i
         return moonep::set_last_error(MOONEP_ERR_INVALID_ARG, kFn,
                                       "topk_idx or a plan output pointer is NULL");
     void* scratch = nullptr;
-    cudaError_t e = scratch_address(&scratch);
+    const char* addr_why = nullptr;
+    cudaError_t e = scratch_address(static_cast<cudaStream_t>(stream), &scratch, &addr_why);
     if (e != cudaSuccess)
-        return moonep::set_last_error(MOONEP_ERR_CUDA, kFn, cudaGetErrorString(e));
+        return moonep::set_last_error(MOONEP_ERR_CUDA, kFn,
+                                      addr_why ? addr_why : cudaGetErrorString(e));
     moonep::PlanLaunch a;
     a.R = c->R; a.S = c->S; a.E = c->E; a.K = c->K; a.B = c->B; a.rule = c->rule;
     a.idx = topk_idx;

@@ -26,7 +26,7 @@ struct Views {
 
 __global__ void __launch_bounds__(THREADS) prefetch_kernel(Views views,
                                                           const int32_t* __restrict__ slot_expert,
-                                                          const int32_t* __restrict__ status,
+                                                          int32_t* status,
                                                           int R, int E, int B, int Er,
                                                           long long row_bytes) {
     if (load_status(status) != MOONEP_STATUS_OK) return;
@@ -36,7 +36,11 @@ __global__ void __launch_bounds__(THREADS) prefetch_kernel(Views views,
         const int slot = (int)(it / pieces);
         const long long piece = it % pieces;
         const int e = __ldg(slot_expert + slot);
-        if (e < 0 || e >= E) continue;
+        if (e < 0) continue;  // unused slot
+        if (e >= E) {         // range guard
+            if (threadIdx.x == 0) report_internal(status);
+            continue;
+        }
         const int r = slot / B, j = slot % B;
         const char* src = views.v[e / Er] + (long long)e * row_bytes + piece * PIECE;
         char* dst = views.v[r] + (long long)(E + j) * row_bytes + piece * PIECE;
@@ -62,7 +66,7 @@ __global__ void __launch_bounds__(THREADS) prefetch_kernel(Views views,
 
 __global__ void __launch_bounds__(THREADS) grad_reduce_kernel(Views views,
                                                              const int32_t* __restrict__ slot_expert,
-                                                             const int32_t* __restrict__ status,
+                                                             int32_t* status,
                                                              int R, int E, int B, int Er,
                                                              long long row_bytes) {
     if (load_status(status) != MOONEP_STATUS_OK) return;
@@ -73,6 +77,7 @@ __global__ void __launch_bounds__(THREADS) grad_reduce_kernel(Views views,
     int* head = nxt + RB; // [RB] 1 if this slot is its expert's first replica
     for (int q = threadIdx.x; q < RB; q += THREADS) {
         const int e = __ldg(slot_expert + q);
+        if (e >= E && blockIdx.x == 0) report_internal(status);  // range guard
         se[q] = (e >= 0 && e < E) ? e : -1;
     }
     __syncthreads();

@@ -36,7 +36,11 @@
  *    out of range, a device wait that gave up) are written by the planner to
  *    the plan's device status block.  Dispatch, combine, prefetch, grad-reduce
  *    and the expert stand-in read it first and do nothing when it is not
- *    MOONEP_STATUS_OK, so a failed plan never moves data.
+ *    MOONEP_STATUS_OK, so a failed plan never moves data.  A kernel that
+ *    finds a plan index outside its buffers (dst_row outside [0, P), a slot
+ *    expert >= E: a corrupted or overwritten plan) skips or clamps that
+ *    access, so nothing outside the buffers is touched, and sets
+ *    MOONEP_STATUS_INTERNAL.
  *  - Layouts are row-major and contiguous.  Row pointers must be 16-byte
  *    aligned (every cudaMalloc / torch allocation is).
  */
@@ -331,9 +335,13 @@ int moonep_weights_destroy(moonep_weights_t* w);
  * every GPU that loads the library holds it until the process exits.  A
  * larger E returns MOONEP_ERR_INVALID_ARG.  The call itself allocates
  * nothing: no cudaMalloc, no cudaFree, no allocating library routine.
- *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress, with that device current) and caches it; make
- *    that first call before any stream capture.
+ *  - Every call made outside a stream capture looks up the array's device
+ *    address (cudaGetSymbolAddress, with the calling device current) and
+ *    caches it per device with the current driver context.  A call inside a
+ *    capture uses that cache and returns MOONEP_ERR_CUDA if it holds no
+ *    address for the current context, so make the first call on a device --
+ *    and the first after a device reset or a change of driver context --
+ *    outside any capture.
  *  - All calls share the one array, which keeps the last call's contents.
  *    Nothing in it needs clearing between calls (each call rewrites every
  *    word it reads; the wait counters live in the plan's status block, which

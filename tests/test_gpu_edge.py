@@ -148,3 +148,74 @@ def test_invalid_arguments_rejected_before_launch():
         m.dispatch(cfg, bufs, x, recv, recv_scale=torch.zeros(4, device="cuda"))
     with pytest.raises(m.MoonEPError, match="aligned"):
         m.dispatch(cfg, bufs, x.view(-1)[1:], recv)
+
+
+@pytest.mark.parametrize("bad", [-1, 1 << 20])
+def test_corrupted_plan_reported_as_internal(bad):
+    """A plan whose dst_row (or slot map) the caller overwrote with an index
+    outside the buffers: every kernel's range check skips or clamps the
+    access and sets MOONEP_STATUS_INTERNAL instead of reporting OK.  The bad
+    values are made on the host; no access leaves its buffer."""
+    m = me()
+    cfgd = wl.cfg_with("fp8", R=2, S=64, E=4, K=2, B=2, H=1024, Hp=1024, alpha=1.5,
+                       payload="bf16")
+    T, P, H = 128, 256, 1024
+    idx, w = wl.routing(cfgd, seed=0)
+    x = wl.hidden(T, H, seed=0).cuda()
+    w_d = torch.from_numpy(w).cuda()
+    idx_d = torch.from_numpy(idx).cuda()
+    bad = bad if bad < 0 else P + bad
+
+    def fresh(payload="bf16"):
+        cfg = m.config_from(dict(cfgd, payload=payload))
+        bufs = m.PlanBuffers(cfg)
+        m.plan(cfg, idx_d, bufs)
+        torch.cuda.synchronize()
+        assert m.plan_status(bufs)[0] == m.STATUS_OK
+        return cfg, bufs
+
+    def corrupt_row(bufs):
+        bufs.dst_row[37] = bad
+        torch.cuda.synchronize()
+
+    recv = torch.zeros((P, H), dtype=torch.bfloat16, device="cuda")
+    y = torch.zeros((T, H), dtype=torch.bfloat16, device="cuda")
+    calls = [
+        lambda cfg, bufs: m.dispatch(cfg, bufs, x, recv),
+        lambda cfg, bufs: m.combine(cfg, bufs, recv, w_d, y),
+        lambda cfg, bufs: m.combine_backward(cfg, bufs, y, recv, w_d, torch.empty_like(recv),
+                                             torch.empty_like(w_d)),
+        lambda cfg, bufs: m.dispatch_backward(cfg, bufs, recv, torch.empty_like(y)),
+    ]
+    for call in calls:
+        cfg, bufs = fresh()
+        corrupt_row(bufs)
+        call(cfg, bufs)
+        assert m.plan_status(bufs)[0] == m.STATUS_INTERNAL
+    # fp8 dispatch
+    cfg, bufs = fresh("fp8")
+    corrupt_row(bufs)
+    q = torch.zeros((P, H), dtype=torch.uint8, device="cuda")
+    sc = torch.zeros((P, H // 128), dtype=torch.float32, device="cuda")
+    m.dispatch(cfg, bufs, x, q, sc)
+    assert m.plan_status(bufs)[0] == m.STATUS_INTERNAL
+    # a slot map entry >= E: prefetch and grad-reduce
+    for kind in ("prefetch", "grad_reduce"):
+        cfg, bufs = fresh()
+        bufs.slot_expert[1] = cfg.E + (0 if bad < 0 else 7)
+        torch.cuda.synchronize()
+        eb = 2 if kind == "prefetch" else 4
+        wv = m.WeightViews(cfg, elem_bytes=eb)
+        try:
+            if kind == "prefetch":
+                m.prefetch(cfg, bufs, wv.ptrs, elem_bytes=2)
+            else:
+                m.grad_reduce(cfg, bufs, wv.ptrs)
+            assert m.plan_status(bufs)[0] == m.STATUS_INTERNAL
+        finally:
+            wv.close()
+    # and an intact plan still reports OK through every call
+    cfg, bufs = fresh()
+    for call in calls:
+        call(cfg, bufs)
+    assert m.plan_status(bufs)[0] == m.STATUS_OK

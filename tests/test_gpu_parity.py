@@ -160,11 +160,18 @@ def test_zipf_sweep(alpha, rule):
         assert o["status"] == 0  # keep-lightest fits the slot budget at every skew
 
 
-@pytest.mark.parametrize("name,rule", [("hot", 0), ("hot", 2), ("hot_tokens", 0), ("hot_tokens", 1)])
-def test_hot_adversarial(name, rule):
+@pytest.mark.parametrize("name,rule,expert", [
+    ("hot", 0, "identity"), ("hot", 0, "scale"), ("hot", 2, "identity"),
+    ("hot_tokens", 0, "identity"), ("hot_tokens", 1, "scale")])
+def test_hot_adversarial(name, rule, expert):
+    """The largest workload.  With the identity expert all K rows of a token
+    hold the same vector, so a combine that gathered the wrong one of them
+    would still agree; the scale expert (1 + e/E per row group) makes every
+    row of a token differ, so the sampled tokens' y also pins which row each
+    (t, k) was gathered from and which weight it was paired with."""
     cfgd = wl.WORKLOADS[name]
     idx, w, x = routing_and_x(cfgd, seed=0)
-    out, o = _check_large(cfgd, idx, w, x, rule, "identity", n_sample=256)
+    out, o = _check_large(cfgd, idx, w, x, rule, expert, n_sample=256)
     assert o["status"] == 0
     if name == "hot":
         assert o["maxvio"] > 100  # half of all picks on one expert
@@ -172,6 +179,19 @@ def test_hot_adversarial(name, rule):
         assert o["expert_count"].max() >= cfgd["R"] * cfgd["S"] // 2  # half the tokens
     del out
     torch.cuda.empty_cache()
+
+
+def test_fp8_workload_scale_expert():
+    """The fp8 workload with the scale expert applied to the dequantised
+    rows: sampled tokens' y bit-exact, so each of a token's K rows is the one
+    its (t, k) was dispatched to."""
+    cfgd = wl.WORKLOADS["fp8"]
+    idx, w, x = routing_and_x(cfgd, seed=0)
+    for rule in (0, 2):
+        out, o = _check_large(cfgd, idx, w, x, rule, "scale", n_sample=256)
+        assert o["status"] == 0
+        del out
+        torch.cuda.empty_cache()
 
 
 def test_fp8_workload():

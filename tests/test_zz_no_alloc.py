@@ -12,7 +12,9 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from dispatch_moonep_plan_b200 import workloads as wl
+from gpu_helpers import compare_plans
 
 pytestmark = pytest.mark.gpu
 
@@ -34,6 +36,10 @@ def _plan_both(m, cfgd, seed, rule, alpha=None):
                                    ctypes.byref(got.c), ctypes.c_void_p(stream.cuda_stream))
     assert rc == m.OK, m.lib.moonep_last_error()
     torch.cuda.synchronize()
+    # the plan stands on its own against the CPU oracle, as well as against
+    # the workspace planner
+    o = oracle.plan(cfgd["R"], cfgd["S"], cfgd["E"], cfgd["K"], cfgd["B"], idx, rule=rule)
+    compare_plans(got.host(), o)
     return ref.host(), got.host()
 
 
@@ -63,6 +69,20 @@ def test_noalloc_matches_plan_on_consecutive_calls():
     r3, g3 = _plan_both(m, wl.WORKLOADS["zipf"], seed=0, rule=0, alpha=1.5)
     _same(r3, g3)
     assert r3["status"] == m.STATUS_SLOT_BUDGET
+
+
+def test_noalloc_at_its_largest_E():
+    """E = MOONEP_NOALLOC_MAX_E fills the static scratch to its last word
+    (per-block tables of E columns for every planner block); E = 384 is the
+    hot-expert workload's expert count.  Both bit-exact, twice in a row."""
+    from dispatch_moonep_plan_b200 import moonep as m
+    assert m.NOALLOC_MAX_E == 512
+    big = dict(name="noalloc512", R=4, S=512, E=512, K=4, B=16, H=64, Hp=0, routing="zipf",
+               alpha=1.0, payload="bf16")
+    mid = dict(big, name="noalloc384", R=32, S=256, E=384, K=8, B=16)
+    for cfgd, rule in ((big, 2), (mid, 1), (big, 0)):
+        r, g = _plan_both(m, cfgd, seed=5, rule=rule)
+        _same(r, g)
 
 
 def test_noalloc_rejects_E_above_its_limit():
