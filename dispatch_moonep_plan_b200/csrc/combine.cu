@@ -56,7 +56,7 @@ __global__ void __launch_bounds__(THREADS) combine_kernel(const uint4* __restric
                                                          uint4* __restrict__ y,
                                                          int32_t* status, int T,
                                                          int K, int H8) {
-    if (load_status(status) != MOONEP_STATUS_OK) return;
+    if (!block_status_ok(status)) return;
     const int lane = threadIdx.x & 31;
     const long long nw = (long long)gridDim.x * WARPS;
     for (long long i = (long long)blockIdx.x * WARPS + (threadIdx.x >> 5); i < T; i += nw) {
@@ -130,7 +130,7 @@ __global__ void __launch_bounds__(THREADS) combine_kfirst_kernel(const uint4* __
                                                                 uint4* __restrict__ y,
                                                                 int32_t* status, int T, int K,
                                                                 int H8) {
-    if (load_status(status) != MOONEP_STATUS_OK) return;
+    if (!block_status_ok(status)) return;
     const int lane = threadIdx.x & 31;
     const long long nw = (long long)gridDim.x * WARPS;
     for (long long i = (long long)blockIdx.x * WARPS + (threadIdx.x >> 5); i < T; i += nw) {
@@ -201,7 +201,7 @@ __global__ void __launch_bounds__(THREADS, 2) combine_bwd_kernel(const uint4* __
                                                              float* __restrict__ d_w,
                                                              int32_t* status, int T, int K,
                                                              int H8) {
-    if (load_status(status) != MOONEP_STATUS_OK) return;
+    if (!block_status_ok(status)) return;
     const int lane = threadIdx.x & 31;
     const int P = T * K;
     const long long nw = (long long)gridDim.x * WARPS;
@@ -284,7 +284,7 @@ __global__ void __launch_bounds__(THREADS) combine_bwd_seq_kernel(const uint4* _
                                                              float* __restrict__ d_w,
                                                              int32_t* status, int T, int K,
                                                              int H8) {
-    if (load_status(status) != MOONEP_STATUS_OK) return;
+    if (!block_status_ok(status)) return;
     const int lane = threadIdx.x & 31;
     const int P = T * K;
     const long long nw = (long long)gridDim.x * WARPS;

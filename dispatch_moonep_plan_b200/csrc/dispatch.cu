@@ -27,7 +27,7 @@ __global__ void __launch_bounds__(THREADS) dispatch_bf16_kernel(const uint4* __r
                                                                int32_t* status, int T, int K,
                                                                int H8) {
     const int P = T * K;
-    if (load_status(status) != MOONEP_STATUS_OK) return;
+    if (!block_status_ok(status)) return;
     const int lane = threadIdx.x & 31;
     const long long nw = (long long)gridDim.x * WARPS;
     for (long long t = (long long)blockIdx.x * WARPS + (threadIdx.x >> 5); t < T; t += nw) {
@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(THREADS) dispatch_fp8_kernel(const uint4* __re
                                                               const int32_t* __restrict__ dst_row,
                                                               int32_t* status, int T, int K,
                                                               int H8) {
-    if (load_status(status) != MOONEP_STATUS_OK) return;
+    if (!block_status_ok(status)) return;
     extern __shared__ float row_scales[];  // [WARPS][H8/16]
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int P = T * K;

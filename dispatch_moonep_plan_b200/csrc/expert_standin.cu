@@ -43,7 +43,7 @@ __global__ void __launch_bounds__(THREADS) expert_kernel(const void* __restrict_
                                                         const int32_t* __restrict__ status,
                                                         int R, int C, int E, int B, int H8,
                                                         int mode, int fp8) {
-    if (load_status(status) != MOONEP_STATUS_OK) return;
+    if (!block_status_ok(status)) return;
     const int lane = threadIdx.x & 31;
     const long long rows = (long long)R * C;
     const long long nw = (long long)gridDim.x * WARPS;

@@ -68,6 +68,20 @@ __device__ __forceinline__ int load_status(const int32_t* status)
     return __ldcg(status + ST_STATUS);
 }
 
+// Whether a kernel may run: the plan's status read once per block.  Kernels
+// of the path can set a failure status while other blocks are starting (a
+// range check reporting INTERNAL, an expert-GEMM wait running out), so
+// threads reading the word on their own could disagree; the block would then
+// split, with some threads gone while the rest wait on shuffles or use
+// shared data those threads were to fill.  Thread 0 reads, the block agrees.
+__device__ __forceinline__ bool block_status_ok(const int32_t* status)
+{
+    __shared__ int st;
+    if (threadIdx.x == 0) st = load_status(status);
+    __syncthreads();
+    return st == MOONEP_STATUS_OK;
+}
+
 // A kernel's own range check found an index outside its buffers (a planner
 // bug, or a plan the caller overwrote): record MOONEP_STATUS_INTERNAL in the
 // status block, unless an earlier failure is already there.  The caller skips

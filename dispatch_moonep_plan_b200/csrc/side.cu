@@ -29,7 +29,7 @@ __global__ void __launch_bounds__(THREADS) prefetch_kernel(Views views,
                                                           int32_t* status,
                                                           int R, int E, int B, int Er,
                                                           long long row_bytes) {
-    if (load_status(status) != MOONEP_STATUS_OK) return;
+    if (!block_status_ok(status)) return;
     const long long pieces = (row_bytes + PIECE - 1) / PIECE;
     const long long items = (long long)R * B * pieces;
     for (long long it = blockIdx.x; it < items; it += gridDim.x) {
@@ -69,7 +69,7 @@ __global__ void __launch_bounds__(THREADS) grad_reduce_kernel(Views views,
                                                              int32_t* status,
                                                              int R, int E, int B, int Er,
                                                              long long row_bytes) {
-    if (load_status(status) != MOONEP_STATUS_OK) return;
+    if (!block_status_ok(status)) return;
     extern __shared__ int sm[];
     const int RB = R * B;
     int* se = sm;         // [RB] slot map
