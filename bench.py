@@ -397,9 +397,13 @@ def run_gpu(args, cfgd, emit=True):
     t_comb = [e[3].elapsed_time(e[4]) for e in evs]
     t_step = [a + b + c for a, b, c in zip(t_plan, t_disp, t_comb)]
     region_ms = region[0].elapsed_time(region[1])
-    m_plan, m_disp, m_comb, m_step = (statistics.mean(v) for v in (t_plan, t_disp, t_comb, t_step))
-    med = dict(plan_us=statistics.median(t_plan) * 1e3, dispatch_us=statistics.median(t_disp) * 1e3,
-               combine_us=statistics.median(t_comb) * 1e3, step_ms=statistics.median(t_step))
+    # per-kernel figures: the median of the K steps (a host stall between two
+    # event records lands in one interval and would move a mean), then the
+    # max over ranks; the means and the slowest step are kept beside them
+    m_plan, m_disp, m_comb, m_step = (statistics.median(v) for v in (t_plan, t_disp, t_comb, t_step))
+    mean = dict(plan_us=statistics.mean(t_plan) * 1e3, dispatch_us=statistics.mean(t_disp) * 1e3,
+                combine_us=statistics.mean(t_comb) * 1e3, step_ms=statistics.mean(t_step),
+                slowest_step_ms=max(t_step))
     m_plan, m_disp, m_comb, m_step, region_ms = reduce_max(
         [m_plan, m_disp, m_comb, m_step, region_ms], world)
 
@@ -446,7 +450,7 @@ def run_gpu(args, cfgd, emit=True):
         dispatch_frac=disp_gbs / peak, combine_frac=comb_gbs / peak,
         maxvio=maxvio, tokens_per_s=world * T / (step_ms * 1e-3),
         step_timing=graph_note, step_ms_per_kernel_events=m_step,
-        region_ms=region_ms, median=med,
+        region_ms=region_ms, stat="median of the K timed steps, max over ranks", mean=mean,
         e2e=dict(value=world * P / (e2e["ms"] * 1e-3), unit=UNIT,
                  h2d_bytes_per_step=e2e["h2d"], d2h_bytes_per_step=e2e["d2h"],
                  ms_per_step=e2e["ms"], serial_ms_per_step=e2e["serial_ms"],
@@ -503,11 +507,12 @@ def graph_step_time(step, flush, args, world, stream):
         b.record(cur)
     torch.cuda.synchronize()
     barrier(world)
-    m = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    m = statistics.median(a.elapsed_time(b) for a, b in evs)
     m = reduce_max([m], world)[0]
     del g
     return m, ("one CUDA graph of plan -> dispatch -> combine per step, CUDA events around "
-               "each replay, L2 flushed before each outside the events")
+               "each replay, L2 flushed before each outside the events; the median of the K "
+               "replays")
 
 
 def e2e_pipelined(me, cfg, bufs, x, idx, w, recv, scale, eo, fp8, args, world):
@@ -622,7 +627,7 @@ def measure_backward(me, cfg, bufs, T, P, H, K, flush, world, eo, reps=10):
             torch.cuda.synchronize()
             if i >= 2:
                 ts.append(a.elapsed_time(b))
-        return reduce_max([statistics.mean(ts)], world)[0]
+        return reduce_max([statistics.median(ts)], world)[0]
 
     tc = timeit(lambda: me.combine_backward(cfg, bufs, dy, eo, w, d_eo, d_w))
     td = timeit(lambda: me.dispatch_backward(cfg, bufs, eo, dx))
@@ -637,7 +642,7 @@ def measure_backward(me, cfg, bufs, T, P, H, K, flush, world, eo, reps=10):
     return out
 
 
-def measure_side(me, wl, flush, world, reps=10, S=None, Hp=None):
+def measure_side(me, wl, flush, world, reps=10, S=None, Hp=None, rule=0):
     """Replica prefetch (bf16 weights) and replica grad-reduce (fp32 grads) at
     the fp8 workload's sizes on VMM-aliased [E+B, H, H'] views (S, if given,
     shrinks only the routing that places the slots; Hp the weight rows)."""
@@ -649,7 +654,7 @@ def measure_side(me, wl, flush, world, reps=10, S=None, Hp=None):
     if Hp:
         kw["Hp"] = Hp
     cfgd = wl.cfg_with("fp8", **kw)
-    cfg = me.config_from(cfgd, 0)
+    cfg = me.config_from(cfgd, rule)
     idx, _ = wl.routing(cfgd, seed=0)
     bufs = me.PlanBuffers(cfg)
     me.plan(cfg, torch.from_numpy(idx).cuda(), bufs)
@@ -675,7 +680,7 @@ def measure_side(me, wl, flush, world, reps=10, S=None, Hp=None):
             torch.cuda.synchronize()
             if i >= 2:
                 ts.append(a.elapsed_time(b))
-        return reduce_max([statistics.mean(ts)], world)[0]
+        return reduce_max([statistics.median(ts)], world)[0]
 
     out = dict(workload=cfgd["name"] + " H'=%d" % Hp, used_slots=n_used,
                replicated_experts=int((reps_per_e > 0).sum()))
@@ -781,8 +786,8 @@ def measure_gemm(me, wl, flush, world, reps=5, S=None, local=None, rule=0, base=
         del w0
     finally:
         views.close()
-    t = reduce_max([statistics.mean(ts)], world)[0]
-    t_c = reduce_max([statistics.mean(tc)], world)[0]
+    t = reduce_max([statistics.median(ts)], world)[0]
+    t_c = reduce_max([statistics.median(tc)], world)[0]
     flops = 2.0 * P * H * Hp
     tf = flops / (t * 1e-3) / 1e12
     tf_c = flops / (t_c * 1e-3) / 1e12
@@ -840,7 +845,7 @@ def measure_gemm_fp8(me, wl, flush, world, reps=5, S=None, local=None, rule=0):
             b.record(stream)
             torch.cuda.synchronize()
             ts.append(a.elapsed_time(b))
-        return reduce_max([statistics.mean(ts)], world)[0]
+        return reduce_max([statistics.median(ts)], world)[0]
 
     views = me.WeightViews(cfg, elem_bytes=2)
     try:
@@ -936,6 +941,9 @@ def main(argv=None):
     ap.add_argument("--backward-only", action="store_true",
                     help="time only the backward of combine and of dispatch on --workload "
                          "(--S shrinks it) and print their line")
+    ap.add_argument("--plan-only", action="store_true",
+                    help="time only the planner on --workload (its inputs and outputs only: "
+                         "a few tens of MB on the device) and print its line")
     ap.add_argument("--sweep", default=None,
                     help="also time every workload / skew and write JSON lines to this file")
     args = ap.parse_args(argv)
@@ -955,6 +963,9 @@ def main(argv=None):
     if args.side_only or args.backward_only:
         run_part_only(args, cfgd)
         return
+    if args.plan_only:
+        run_plan_only(args, cfgd)
+        return
     out = run_gpu(args, cfgd)
     if out is not None and int(os.environ.get("WORLD_SIZE", "1")) == 1 and not args.no_sweep:
         out["sweep"] = skew_sweep(args)
@@ -963,6 +974,40 @@ def main(argv=None):
         print(json.dumps(out), flush=True)
     if args.sweep and out is not None:
         run_sweep(args)
+
+
+def run_plan_only(args, cfgd):
+    """The planner alone on the workload's full routing: CUDA events around
+    each call (status memset + one cooperative kernel), L2 flushed before
+    each outside the events."""
+    import torch
+
+    from dispatch_moonep_plan_b200 import moonep as me
+    from dispatch_moonep_plan_b200 import workloads as wl
+    flush_w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    cfg = me.config_from(cfgd, args.rule)
+    idx, _ = wl.routing(cfgd, seed=0, alpha=args.alpha)
+    idx_d = torch.from_numpy(idx).cuda()
+    bufs = me.PlanBuffers(cfg)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        flush_w.zero_()
+        me.plan(cfg, idx_d, bufs, stream)
+    torch.cuda.synchronize()
+    st = me.plan_status(bufs)
+    ts = []
+    for _ in range(args.steps):
+        flush_w.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        me.plan(cfg, idx_d, bufs, stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b) * 1e3)
+    print(json.dumps(dict(plan=dict(workload=cfgd["name"], rule=args.rule, status=st,
+                                    maxvio=float(bufs.maxvio.item()),
+                                    plan_us=statistics.median(ts), mean_us=statistics.mean(ts),
+                                    min_us=min(ts), calls=len(ts)))), flush=True)
 
 
 def run_part_only(args, cfgd):
@@ -979,7 +1024,7 @@ def run_part_only(args, cfgd):
 
     if args.side_only:
         print(json.dumps(dict(side=measure_side(me, wl, flush, 1, reps=args.steps, S=args.S,
-                                                Hp=args.Hp))), flush=True)
+                                                Hp=args.Hp, rule=args.rule))), flush=True)
         return
     cfg = me.config_from(dict(cfgd, payload="bf16"), args.rule)
     s = me.sizes(cfg)
