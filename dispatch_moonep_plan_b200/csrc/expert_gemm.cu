@@ -17,14 +17,16 @@
 //    (K-major), B = 64 x BN of the weight row (H' contiguous, MN-major), both
 //    128-byte swizzled in shared memory;
 //  - fp8 payload: A never exists in bf16 outside the SM.  Warp 6 streams the
-//    e4m3 tiles into a ring of 8 slots, 8 converter warps widen them
+//    e4m3 tiles into a ring of 4 slots, 8 converter warps widen them
 //    (a = bf16(float(q) * scale)) straight into tensor memory with
 //    tcgen05.st, and the MMA reads A from there; shared memory then holds
-//    only B.  Tiles are 128 x 192, so two accumulators (384 columns) and 4 A
-//    stages (32 columns each) fill the 512 columns; the last n-tile may be
-//    partial;
-//  - the fp32 accumulator lives in tensor memory, two buffers of BN columns,
-//    so the epilogue of one tile overlaps the main loop of the next;
+//    only B.  A tile is 128 x 384: each widened A block feeds two MMAs of
+//    N = 192, so A is widened once per 384 output columns (4 times per row
+//    block at H' = 1536, not 8).  One 384-column accumulator and 3 A stages
+//    (32 columns each) fit the 512 columns; the last n-tile may be partial;
+//  - the fp32 accumulator lives in tensor memory; the bf16 payload keeps two
+//    buffers of BN columns, so the epilogue of one tile overlaps the main
+//    loop of the next (the fp8 payload's single buffer does not);
 //  - the epilogue reads 32 lanes x 32 columns per tcgen05.ld, rounds once to
 //    bf16 (round-to-nearest-even) and stores only the rows of the group.
 //
@@ -236,25 +238,30 @@ struct GemmArgs {
     int debug_stall;  // epilogue waits on a barrier nothing completes
 };
 
-template <int BN, int STAGES, bool FP8A, int CW, int A8_SLOTS>
+template <int BN, int STAGES, bool FP8A, int CW, int A8_SLOTS, int NSUB>
 __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
     expert_gemm_kernel(const __grid_constant__ CUtensorMap tmX,
                        const __grid_constant__ CUtensorMap tmW, GemmArgs p) {
     constexpr int THREADS = threads_for<FP8A, CW>();
-    constexpr int B_BYTES = BK * BN * 2;
+    // a tile is BM rows x TN = NSUB * BN columns: NSUB MMAs of N = BN per
+    // k-step share one A block (fp8 payload: A is widened once per TN columns)
+    constexpr int TN = NSUB * BN;
+    constexpr int B_BYTES = BK * TN * 2;
     // a stage of the MMA ring: bf16 A (SW128, K-major) | B.  fp8 payload: A
     // lives in tensor memory, so a stage holds only B, and the e4m3 tiles
     // land in their own ring of A8_SLOTS after the stages.
     constexpr int STAGE_A = FP8A ? 0 : A_BYTES;
     constexpr int STAGE_BYTES = STAGE_A + B_BYTES;
     constexpr int A8S = FP8A ? A8_SLOTS : 0;
-    // two accumulators of BN columns; fp8 payload: then A stage s at columns
-    // ACOL + 32 s (128 rows x 64 bf16, two elements per column)
-    constexpr int ACOL = 2 * BN;
-    constexpr int TMEM_COLS = FP8A ? 512 : 2 * BN;
-    static_assert(!FP8A || (ACOL + 32 * STAGES <= 512 && CW % 4 == 0 && CW <= 16),
-                  "fp8 payload: two accumulators and the A stages in 512 columns, whole "
-                  "converter warps per lane quarter");
+    // NACC accumulators of TN columns (two, so that the epilogue of one tile
+    // overlaps the next tile's main loop, when they fit); fp8 payload: then A
+    // stage s at columns ACOL + 32 s (128 rows x 64 bf16, two per column)
+    constexpr int NACC = (FP8A ? 2 * TN + 32 * STAGES : 2 * TN) <= 512 ? 2 : 1;
+    constexpr int ACOL = NACC * TN;
+    constexpr int TMEM_COLS = FP8A ? 512 : NACC * TN;
+    static_assert(NACC * TN + (FP8A ? 32 * STAGES : 0) <= 512 && TN <= 512,
+                  "accumulators (and fp8 A stages) in the 512 tensor-memory columns");
+    static_assert(!FP8A || (CW % 4 == 0 && CW <= 16), "whole converter warps per lane quarter");
     // k-block of A: 128 rows x 128 B; one k-step (16 elements) = 32 B along a row.
     // k-block of B: BN/64 column chunks of 64 k-rows x 128 B (8 KiB each); one
     // k-step = 16 k-rows = 2 KiB; the next 64-column chunk is 8 KiB further.
@@ -267,7 +274,7 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
     uint64_t* a8full = conv + STAGES;   // fp8 payload: e4m3 tile landed [A8_SLOTS]
     uint64_t* a8empty = a8full + A8_SLOTS;  // fp8 payload: e4m3 tile read [A8_SLOTS]
     uint64_t* tfull = a8empty + A8_SLOTS;
-    uint64_t* tempty = tfull + 2;
+    uint64_t* tempty = tfull + 2;  // [NACC] (two slots kept either way)
     uint64_t* drain = tempty + 2;
     uint64_t* never = drain + 1;
     uint32_t* tmem_slot = (uint32_t*)(never + 1);
@@ -286,7 +293,7 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
     const int G = p.E + p.B;      // groups per rank
     const int per = p.Er + p.B;   // groups a plan can fill per rank
     const int npairs = p.R * per;
-    const int ntn = (p.Hp + BN - 1) / BN;  // the last n-tile may be partial
+    const int ntn = (p.Hp + TN - 1) / TN;  // the last n-tile may be partial
     const int kblocks = p.H / BK;
 
     if (tid == 0) {
@@ -386,7 +393,7 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
                 // 64-column boxes of B inside H' (all of them unless the
                 // last n-tile is partial; the rest of the stage is not read
                 // into any stored column)
-                const int nbox = min(BN / 64, (p.Hp - nt * BN) / 64);
+                const int nbox = min(TN / 64, (p.Hp - nt * TN) / 64);
                 bool ok = true;
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait(&empty[s], ph ^ 1, p.wait_ns, &abort_flag)) {
@@ -402,9 +409,9 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
                         tma_load_2d(a, &tmX, &full[s], kb * BK, row0);
                     }
 #pragma unroll
-                    for (int j = 0; j < BN / 64; ++j)
+                    for (int j = 0; j < TN / 64; ++j)
                         if (j < nbox)
-                            tma_load_2d(b + j * 8192, &tmW, &full[s], nt * BN + 64 * j,
+                            tma_load_2d(b + j * 8192, &tmW, &full[s], nt * TN + 64 * j,
                                         wrow0 + kb * BK);
                     ++issued;
                     if (++s == STAGES) {
@@ -436,7 +443,11 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
             for (int tile = blockIdx.x; tile < total && !abort_flag; tile += gridDim.x) {
                 if (!mbar_wait(&tempty[acc], acc_ph ^ 1, p.wait_ns, &abort_flag)) break;
                 asm volatile("tcgen05.fence::after_thread_sync;");
-                const uint32_t d = tmem + acc * BN;
+                const uint32_t d = tmem + acc * TN;
+                // sub-tiles wholly past H' (a partial last n-tile) are skipped
+                int nt_, pair_, mt_;
+                locate(tile, pair_, mt_, nt_);
+                const int nsub = min(NSUB, (p.Hp - nt_ * TN + BN - 1) / BN);
                 bool ok = true;
                 for (int kb = 0; kb < kblocks; ++kb) {
                     // the TMA loads landed; fp8: and the converter warps have
@@ -451,13 +462,21 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
                     const uint32_t b = a + STAGE_A;
 #pragma unroll
                     for (int ks = 0; ks < BK / 16; ++ks) {
-                        if constexpr (FP8A)
-                            mma_bf16_tmem_a(d, tmem + ACOL + s * 32 + ks * 8,
-                                            sdesc(b + ks * 2048, 8192, 1024), idesc,
-                                            (kb | ks) ? 1u : 0u);
-                        else
-                            mma_bf16(d, sdesc(a + ks * 32, 16, 1024),
-                                     sdesc(b + ks * 2048, 8192, 1024), idesc, (kb | ks) ? 1u : 0u);
+#pragma unroll
+                        for (int sub = 0; sub < NSUB; ++sub) {
+                            if (sub >= nsub) break;
+                            // sub-tile sub: columns sub*BN.. of the accumulator and
+                            // B chunks sub*BN/64.. of the stage
+                            const uint32_t bsub = b + sub * (BN / 64) * 8192;
+                            if constexpr (FP8A)
+                                mma_bf16_tmem_a(d + sub * BN, tmem + ACOL + s * 32 + ks * 8,
+                                                sdesc(bsub + ks * 2048, 8192, 1024), idesc,
+                                                (kb | ks) ? 1u : 0u);
+                            else
+                                mma_bf16(d + sub * BN, sdesc(a + ks * 32, 16, 1024),
+                                         sdesc(bsub + ks * 2048, 8192, 1024), idesc,
+                                         (kb | ks) ? 1u : 0u);
+                        }
                     }
                     any = true;
                     mma_commit(&empty[s]);
@@ -468,7 +487,7 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
                 }
                 if (!ok) break;
                 mma_commit(&tfull[acc]);
-                if (++acc == 2) {
+                if (++acc == NACC) {
                     acc = 0;
                     acc_ph ^= 1;
                 }
@@ -493,11 +512,11 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
             asm volatile("tcgen05.fence::after_thread_sync;");
             const int row_in = mt * BM + q * 32 + lane;
             const bool valid = glo + row_in < ghi;
-            uint16_t* yrow = p.y + (size_t)(r * p.C + glo + row_in) * p.Hp + nt * BN;
-            const uint32_t tbase = tmem + acc * BN + ((uint32_t)(q * 32) << 16);
+            uint16_t* yrow = p.y + (size_t)(r * p.C + glo + row_in) * p.Hp + nt * TN;
+            const uint32_t tbase = tmem + acc * TN + ((uint32_t)(q * 32) << 16);
 #pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 32) {
-                if (nt * BN + c0 >= p.Hp) break;  // partial last n-tile (warp-uniform)
+            for (int c0 = 0; c0 < TN; c0 += 32) {
+                if (nt * TN + c0 >= p.Hp) break;  // partial last n-tile (warp-uniform)
                 uint32_t v[32];
                 asm volatile(
                     "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,"
@@ -526,7 +545,7 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
             asm volatile("tcgen05.fence::before_thread_sync;");
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[acc]);
-            if (++acc == 2) {
+            if (++acc == NACC) {
                 acc = 0;
                 acc_ph ^= 1;
             }
@@ -688,7 +707,7 @@ size_t smem_bytes(int bn, int stages, int npairs, bool fp8a, int a8_slots = 2) {
            (size_t)(3 * stages + 2 * a8_slots + 6) * 8 + 8 + 32 * 4 + (size_t)(npairs + 1) * 4;
 }
 
-template <int BN, int STAGES, bool FP8A, int CW = 8, int A8_SLOTS = 2>
+template <int BN, int STAGES, bool FP8A, int CW = 8, int A8_SLOTS = 2, int NSUB = 1>
 cudaError_t launch_variant(const CUtensorMap& x, const CUtensorMap& w, const GemmArgs& a,
                            size_t smem, int grid, cudaStream_t s) {
     static std::mutex mu;
@@ -699,13 +718,13 @@ cudaError_t launch_variant(const CUtensorMap& x, const CUtensorMap& w, const Gem
     {
         std::lock_guard<std::mutex> lock(mu);
         if (dev < 0 || dev >= 64 || set[dev] < smem) {
-            e = cudaFuncSetAttribute(expert_gemm_kernel<BN, STAGES, FP8A, CW, A8_SLOTS>,
+            e = cudaFuncSetAttribute(expert_gemm_kernel<BN, STAGES, FP8A, CW, A8_SLOTS, NSUB>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return e;
             if (dev >= 0 && dev < 64) set[dev] = smem;
         }
     }
-    expert_gemm_kernel<BN, STAGES, FP8A, CW, A8_SLOTS>
+    expert_gemm_kernel<BN, STAGES, FP8A, CW, A8_SLOTS, NSUB>
         <<<grid, threads_for<FP8A, CW>(), smem, s>>>(x, w, a);
     return cudaGetLastError();
 }
@@ -714,10 +733,15 @@ cudaError_t launch_variant(const CUtensorMap& x, const CUtensorMap& w, const Gem
 
 int expert_gemm_npairs(const moonep_config& c) { return c.R * (c.E / c.R + c.B); }
 
+// fp8 payload: tile columns, MMA-ring stages and e4m3 slots
+constexpr int FP8_TN = 384;
+constexpr int FP8_STAGES = 3;
+constexpr int FP8_A8 = 4;
+
 // the fp8 kernel's configuration, or the smallest bf16 one
 bool expert_gemm_fits(const moonep_config& c) {
     const int np = expert_gemm_npairs(c);
-    return (c.payload == MOONEP_PAYLOAD_FP8 ? smem_bytes(192, 4, np, true, 8)
+    return (c.payload == MOONEP_PAYLOAD_FP8 ? smem_bytes(FP8_TN, FP8_STAGES, np, true, FP8_A8)
                                             : smem_bytes(128, 3, np, false)) <= (size_t)SMEM_LIMIT;
 }
 
@@ -752,9 +776,10 @@ cudaError_t launch_expert_gemm(const moonep_config& c, const moonep_plan_t& p, c
     a.wait_ns = current_wait_limit_ns();
     a.debug_stall = current_barrier_extra() != 0;
     const int grid = device_sm_count();
-    if (fp8)  // 128 x 192 tiles: two accumulators and 4 A stages fill the 512 TMEM columns
-        return launch_variant<192, 4, true, 8, 8>(tx, tw, a, smem_bytes(192, 4, np, true, 8), grid,
-                                                  s);
+    if (fp8)  // 128 x 384 tiles (two MMAs of N = 192 per widened A block): one
+              // accumulator and 3 A stages in the 512 TMEM columns
+        return launch_variant<192, FP8_STAGES, true, 8, FP8_A8, FP8_TN / 192>(
+            tx, tw, a, smem_bytes(FP8_TN, FP8_STAGES, np, true, FP8_A8), grid, s);
     if (c.Hp % 256 == 0) {
         if (smem_bytes(256, 4, np, false) <= (size_t)SMEM_LIMIT)
             return launch_variant<256, 4, false>(tx, tw, a, smem_bytes(256, 4, np, false), grid, s);
