@@ -189,3 +189,58 @@ def test_rule2_needs_fewer_slots_on_the_workloads(oracle_mod):
             check_plan_invariants(pl, idx, R, S, E, K, 64, rule)
             need.append(int((pl["slot_expert"] >= 0).sum(axis=1).max()))
         assert tuple(need) == want, (name, need)
+
+
+def test_minimum_slot_count_pinned_by_enumeration():
+    """The integer program for the fewest slots any plan can need agrees
+    with an enumeration of every keep/hand-on split on tiny cases."""
+    from slot_optimum import brute_min_max_slots, min_max_slots
+    rng = np.random.default_rng(17)
+    seen = set()
+    for _ in range(200):
+        R = int(rng.integers(2, 4))
+        Er = int(rng.integers(1, 3))
+        C = int(rng.integers(2, 6))
+        cnt = rng.multinomial(R * C, rng.dirichlet(np.full(R * Er, 0.5)))
+        v = min_max_slots(cnt, R, C)
+        assert v == brute_min_max_slots(cnt, R, C), (cnt, R, C)
+        seen.add(v)
+    assert {0, 1, 2} <= seen
+
+
+@pytest.mark.parametrize("rule", [0, 1, 2])
+def test_rules_against_the_minimum_slot_count(oracle_mod, rule):
+    """Every rule's plan is one of the plans the minimum ranges over, so its
+    largest slot count is never below it; on tiny routings rules 1 and 2 stay
+    within two slots of it."""
+    from slot_optimum import min_max_slots, plan_max_slots
+    rng = np.random.default_rng(23 + rule)
+    gap = []
+    for it in range(120):
+        cfg = wl.random_small_cfg(rng)
+        R, S, E, K = cfg["R"], cfg["S"], cfg["E"], cfg["K"]
+        idx, _ = wl.routing(cfg, seed=it)
+        pl = oracle_mod.plan(R, S, E, K, E, idx, rule=rule)
+        assert pl["status"] == 0
+        got = plan_max_slots(pl, E)
+        opt = min_max_slots(np.bincount(idx.reshape(-1), minlength=E), R, S * K)
+        assert got >= opt
+        gap.append(got - opt)
+    if rule >= 1:
+        assert max(gap) <= 2
+
+
+def test_rule2_near_the_minimum_on_the_workloads(oracle_mod):
+    """At the workloads' sizes (seed 0) the fewest slots any plan needs is 2
+    or 3; rule 2 (largest overflow to largest deficit) needs at most one more,
+    rule 0 up to 17."""
+    from slot_optimum import min_max_slots, plan_max_slots
+    for name, alpha in (("zipf", 0.5), ("zipf", 1.0), ("hot", None), ("fp8", None),
+                        ("uniform", None)):
+        c = wl.WORKLOADS[name]
+        R, S, E, K = c["R"], c["S"], c["E"], c["K"]
+        idx, _ = wl.routing(c, seed=0, alpha=alpha)
+        opt = min_max_slots(np.bincount(idx.reshape(-1), minlength=E), R, S * K)
+        assert opt in (2, 3)
+        got = [plan_max_slots(oracle_mod.plan(R, S, E, K, E, idx, rule=r), E) for r in (0, 2)]
+        assert got[0] >= opt and opt <= got[1] <= opt + 1, (name, opt, got)
