@@ -12,9 +12,13 @@
 // Kernel structure (one block per SM, 1024 threads, cooperative launch so
 // that every block is resident and the grid-wide wait cannot deadlock):
 //   A. each block owns a contiguous run of picks, each warp a contiguous part
-//      of it; every warp counts its picks per expert in a private shared
-//      histogram (shared atomics: the order of the counts does not matter
-//      here); the block writes its row hist[block][e].
+//      of it; every warp takes its picks 32 at a time in (t, k) order, finds
+//      the lanes holding the same expert (match.any), and the lowest of them
+//      adds their number to the warp's shared histogram; the count it finds
+//      there (the expert's picks in the warp's earlier rows) plus the lane's
+//      rank among them is the pick's position among the warp's picks of that
+//      expert, kept beside the pick in shared memory; the block writes its
+//      row hist[block][e].
 //   -- one grid-wide wait --
 //   B. every block reads all rows of hist (16-byte loads when E % 4 == 0):
 //      the per-expert totals, and the counts of the blocks before it (its
@@ -22,15 +26,15 @@
 //   C. every block computes the small O(E + R) balance step itself from the
 //      totals (no further grid-wide wait is needed); block 0 writes the
 //      per-layer outputs, each block writes cu_seqlens / slot_expert of the
-//      ranks it owns; then every warp walks its picks again, 32 at a time, in
-//      (t, k) order; the lanes holding the same expert are found with one
-//      ballot per bit of the expert index, and a pick's rank among them is
-//      the count of lower lanes.  A warp's running per-expert offsets start
-//      at the block's offset plus the counts of the block's earlier warps, so
-//      the placement is stable and deterministic without ordered atomics.
-//      (In this kernel the ballots and match_any time the same.)  The
-//      positions are looked up in per-expert tables so that the rest of the
-//      walk is a few shared loads.
+//      ranks it owns; then every warp walks its picks again: a pick's position
+//      among all picks of its expert is the block's offset plus the counts of
+//      the block's earlier warps plus its position within the warp, so the
+//      placement is stable and deterministic without ordered atomics, and the
+//      picks of a row are placed independently.  The destination comes from
+//      one 16-byte per-expert table entry (kept rows) or a short search of
+//      the receiving segments (overflow rows).  When a block's picks do not
+//      fit in shared memory, the walk reads them again and recomputes the
+//      positions row by row with running per-warp offsets.
 // The wait is bounded (globaltimer); when it runs out the block records
 // MOONEP_STATUS_TIMEOUT and returns.
 #include <algorithm>
@@ -78,9 +82,10 @@ struct Smem {
     int* nzri;    // [E+1] items with overflow before each position
     int* ose;     // [E]   start of each expert's rows in the overflow stream
     int* nzlist;  // [E]   experts with overflow, in stream order
-    int* kbase;   // [E]   destination row of the expert's first kept pick
-    int* rlo;     // [E]   first rank receiving the expert's overflow
-    int* rhi;     // [E]   last rank receiving the expert's overflow
+    int4* tab;    // [E]   per expert: rows kept, destination row of its first kept
+                  //       pick, overflow-stream index of pick 0 (ose - kept), picks
+    int* rng;     // [E]   positions of the receiving order that take the expert's
+                  //       overflow: first | last << 16
     int* kept;    // [R]
     int* def;     // [R] C - kept
     int* segs;    // [R] start of the rank's segment in the stream
@@ -90,12 +95,13 @@ struct Smem {
     int* rload;   // [R] home rows before balancing
     int* recv_at; // [R] the rank at each position of the receiving order
     int* sege_at; // [R] segment end at each position of the receiving order
+    int* rbase;   // [R] destination row of stream index 0 at each receiving position
     int* scratch; // [2*SCAN_N*32 + 8]
     int* stash;   // [chunk] the block's picks (when stashed)
 };
 
 __host__ __device__ inline size_t smem_ints(int E, int R) {
-    return (size_t)NW * E + 11 * (size_t)E + 3 + 4 * ((size_t)E + 1) + 9 * (size_t)R +
+    return (size_t)NW * E + 13 * (size_t)E + 3 + 4 * ((size_t)E + 1) + 10 * (size_t)R +
            2 * SCAN_N * 32 + 8;
 }
 
@@ -103,6 +109,7 @@ __device__ inline Smem carve(int* base, int E, int R) {
     Smem s;
     int* p = base;
     s.ov = p; p += (E + 3) & ~3;  // first and padded: read four at a time
+    s.tab = reinterpret_cast<int4*>(p); p += 4 * E;  // 16-byte aligned after ov
     s.whist = p; p += NW * E;
     s.cnt = p; p += E;
     s.bcnt = p; p += E;
@@ -115,9 +122,7 @@ __device__ inline Smem carve(int* base, int E, int R) {
     s.osi = p; p += E + 1;
     s.nzri = p; p += E + 1;
     s.ose = p; p += E;
-    s.kbase = p; p += E;
-    s.rlo = p; p += E;
-    s.rhi = p; p += E;
+    s.rng = p; p += E;
     s.kept = p; p += R;
     s.def = p; p += R;
     s.segs = p; p += R;
@@ -127,6 +132,7 @@ __device__ inline Smem carve(int* base, int E, int R) {
     s.rload = p; p += R;
     s.recv_at = p; p += R;
     s.sege_at = p; p += R;
+    s.rbase = p; p += R;
     s.scratch = p; p += 2 * SCAN_N * 32 + 8;
     s.stash = p;
     return s;
@@ -356,22 +362,28 @@ __device__ int balance(const PlanParams& p, Smem& s, int* misc) {
     return misc[0] >= 0 ? MOONEP_STATUS_SLOT_BUDGET : MOONEP_STATUS_OK;
 }
 
-// Destination row of the pick at position pos among expert e's picks, or -1.
-__device__ __forceinline__ int place(const PlanParams& p, const Smem& s, int e, int pos) {
-    const int k = s.kk[e];
-    if (pos < k) return s.kbase[e] + pos;
-    const int sidx = s.ose[e] + pos - k;
-    // the receiving position lies in [rlo, rhi] of the receiving order
-    int lo = s.rlo[e], hi = s.rhi[e] + 1;
+// Destination row of the pick at position pos among expert e's picks (t =
+// the expert's table entry), or -1 if its stream index is past every segment.
+__device__ __forceinline__ int place(const PlanParams& p, const Smem& s, int e, const int4& t,
+                                     int pos) {
+    if (pos < t.x) return t.y + pos;  // kept on the home rank
+    const int sidx = t.z + pos;       // index in the overflow stream
+    // the receiving position lies in [first, last] of the receiving order
+    const int rr = s.rng[e];
+    int lo = rr & 0xffff, hi = (rr >> 16) + 1;
     while (lo < hi) {
         const int mid = (lo + hi) >> 1;
         if (s.sege_at[mid] <= sidx) lo = mid + 1;
         else hi = mid;
     }
     if (lo >= p.R) return -1;
-    const int rho = s.recv_at[lo];
-    return rho * p.C + s.kept[rho] + (sidx - s.segs[rho]);
+    return s.rbase[lo] + sidx;
 }
+
+// Pack a pick for the walk: its expert (< 2^10) and its position among the
+// warp's picks of that expert (< 2^21: a warp holds at most P / (G * 32) + 1
+// < 2^31 / (148 * 32) + 1 picks).
+__device__ __forceinline__ int pack_pick(int e, int off) { return e | (off << 10); }
 
 __global__ void __launch_bounds__(THREADS, 1) plan_kernel(PlanParams p) {
     extern __shared__ __align__(16) int smem_raw[];
@@ -397,6 +409,7 @@ __global__ void __launch_bounds__(THREADS, 1) plan_kernel(PlanParams p) {
     if (tid == 0) max_count = 0;
     __syncthreads();
     int bad = 0;
+    const unsigned lt_mask = (1u << lane) - 1u;
     for (long long base = wlo; base < whi; base += 32 * UNR) {
         int ev[UNR];
 #pragma unroll
@@ -406,12 +419,24 @@ __global__ void __launch_bounds__(THREADS, 1) plan_kernel(PlanParams p) {
         }
 #pragma unroll
         for (int u = 0; u < UNR; ++u) {
-            const long long q = base + u * 32 + lane;
-            if (q < whi) {
+            if (base + u * 32 < whi) {  // warp-uniform: the row has picks
+                const long long q = base + u * 32 + lane;
+                const bool valid = q < whi;
                 const int e = ev[u];
-                if (p.stash) s.stash[q - clo] = e;
-                if (e < 0 || e >= E) bad = 1;
-                else atomicAdd(wh + e, 1);
+                const bool ok = valid && e >= 0 && e < E;
+                if (valid && !ok) bad = 1;
+                // lanes of the row holding the same expert; every other lane
+                // (no pick, or a bad index) shares the key -1
+                const unsigned peers = __match_any_sync(0xffffffffu, ok ? e : -1);
+                const int rank = __popc(peers & lt_mask);
+                // the lowest lane adds the group's picks; the count it found
+                // is the group's position in the warp's picks of the expert.
+                // The next row's adds come after this one (shuffle, then the
+                // warp's memory-ordering barrier).
+                const int before = (ok && rank == 0) ? atomicAdd(wh + e, __popc(peers)) : 0;
+                const int off = __shfl_sync(0xffffffffu, before, __ffs(peers) - 1) + rank;
+                __syncwarp();
+                if (ok && p.stash) s.stash[q - clo] = pack_pick(e, off);
             }
         }
     }
@@ -546,41 +571,51 @@ __global__ void __launch_bounds__(THREADS, 1) plan_kernel(PlanParams p) {
             run += t;
         }
         const int first = (e / Er) * Er;
-        s.kbase[e] = (e / Er) * p.C + (s.pk[e] - s.pk[first]);
+        const int k = s.kk[e];
+        s.tab[e] = make_int4(k, (e / Er) * p.C + (s.pk[e] - s.pk[first]), s.ose[e] - k, s.cnt[e]);
         const int o = s.ov[e];
-        s.rlo[e] = o > 0 ? upper_bound(s.sege_at, R, s.ose[e]) : 0;
-        s.rhi[e] = o > 0 ? upper_bound(s.sege_at, R, s.ose[e] + o - 1) : 0;
+        s.rng[e] = o > 0 ? upper_bound(s.sege_at, R, s.ose[e]) |
+                               (upper_bound(s.sege_at, R, s.ose[e] + o - 1) << 16)
+                         : 0;
+    }
+    for (int i = tid; i < R; i += THREADS) {
+        const int rho = s.recv_at[i];
+        s.rbase[i] = rho * p.C + s.kept[rho] - s.segs[rho];
     }
     __syncthreads();
 
-    const unsigned lt_mask = (1u << lane) - 1u;
-    const int ebits = E > 1 ? 32 - __clz(E - 1) : 0;  // bits of an expert index
     int internal = 0;
     for (long long base = wlo; base < whi; base += 32 * UNR) {
         const int nu = (int)min((long long)UNR, (whi - base + 31) / 32);  // warp-uniform
-        int ev[UNR];
+        int ev[UNR], pos[UNR];
+        if (p.stash) {
+            // positions within the warp were found in phase A
 #pragma unroll
-        for (int u = 0; u < UNR; ++u) {
-            const long long q = base + u * 32 + lane;
-            ev[u] = q < whi ? (p.stash ? s.stash[q - clo] : __ldg(p.idx + q)) : -1;
-        }
-        int pos[UNR];
+            for (int u = 0; u < UNR; ++u) {
+                const long long q = base + u * 32 + lane;
+                const int v = q < whi ? s.stash[q - clo] : -1;
+                ev[u] = v >= 0 ? (v & 1023) : -1;
+                pos[u] = v >= 0 ? wh[v & 1023] + (v >> 10) : 0;
+            }
+        } else {
+            // picks not kept: read them again, match each row and advance the
+            // warp's running offsets row by row
 #pragma unroll
-        for (int u = 0; u < UNR; ++u) {
-            if (u < nu) {
-                const int e = ev[u];
-                // lanes holding the same expert: one ballot per bit of the
-                // expert index; lanes without a pick (e = -1) match none
-                unsigned peers = __ballot_sync(0xffffffffu, e >= 0);
-                for (int bit = 0; bit < ebits; ++bit) {
-                    const bool set = (e >> bit) & 1;
-                    const unsigned m = __ballot_sync(0xffffffffu, set);
-                    peers &= set ? m : ~m;
+            for (int u = 0; u < UNR; ++u) {
+                const long long q = base + u * 32 + lane;
+                ev[u] = q < whi ? __ldg(p.idx + q) : -1;
+            }
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                if (u < nu) {
+                    const int e = ev[u];
+                    const unsigned peers = __match_any_sync(0xffffffffu, e);
+                    const int run = e >= 0 ? wh[e] : 0;
+                    pos[u] = run + __popc(peers & lt_mask);
+                    __syncwarp();
+                    if (e >= 0 && lane == __ffs(peers) - 1) wh[e] = run + __popc(peers);
+                    __syncwarp();
                 }
-                if (e >= 0) pos[u] = wh[e] + __popc(peers & lt_mask);
-                __syncwarp();
-                if (e >= 0 && lane == __ffs(peers) - 1) wh[e] += __popc(peers);
-                __syncwarp();
             }
         }
 #pragma unroll
@@ -588,8 +623,9 @@ __global__ void __launch_bounds__(THREADS, 1) plan_kernel(PlanParams p) {
             const int e = ev[u];
             if (u < nu && e >= 0) {
                 const long long q = base + u * 32 + lane;
-                const int dst = place(p, s, e, pos[u]);
-                if (dst >= 0 && dst < p.P && pos[u] < s.cnt[e]) {
+                const int4 t = s.tab[e];
+                const int dst = place(p, s, e, t, pos[u]);
+                if (dst >= 0 && dst < p.P && pos[u] < t.w) {
                     p.dst_row[q] = dst;
                     p.src_of_row[dst] = (int)q;
                 } else {
