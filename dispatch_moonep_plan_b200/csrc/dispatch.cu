@@ -64,19 +64,23 @@ __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
     return (uint32_t)r;
 }
 
-// fp8: each lane owns 16 consecutive elements (a "unit", two 16-byte loads);
-// 8 lanes make one 128-element block, so the block amax is 3 xor-shuffles.  A
-// lane's 16 codes leave as one 16-byte store per destination row.  The
-// scales of a row are collected in shared memory (one float per block) and
-// written as one contiguous run per destination row once the row is done.
-// H % 128 == 0, so a row has a whole number of 8-lane blocks.
-template <int U>
+// fp8: each lane owns units of 16 consecutive elements (two 16-byte loads
+// each); 8 lanes make one 128-element block, so the block amax is 3
+// xor-shuffles.  A lane first loads L units of the row (2L loads in flight),
+// then quantises and stores them G units at a time: its 16 codes of a unit
+// leave as one 16-byte store per destination row.  While a token is being
+// quantised, the warp's next token is requested into L2.  The scales of a row
+// are collected in shared memory (one float per block) and written as one
+// contiguous run per destination row once the row is done.  H % 128 == 0, so
+// a row has a whole number of 8-lane blocks.
+template <int L, int G>
 __global__ void __launch_bounds__(THREADS) dispatch_fp8_kernel(const uint4* __restrict__ x,
                                                               uint8_t* __restrict__ recv,
                                                               float* __restrict__ recv_scale,
                                                               const int32_t* __restrict__ dst_row,
                                                               int32_t* status, int T, int K,
                                                               int H8) {
+    static_assert(L % G == 0, "whole groups");
     if (!block_status_ok(status)) return;
     extern __shared__ float row_scales[];  // [WARPS][H8/16]
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -90,51 +94,68 @@ __global__ void __launch_bounds__(THREADS) dispatch_fp8_kernel(const uint4* __re
         const int myrow = lane < K ? __ldg(dst_row + t * K + lane) : 0;
         if (lane < K && (unsigned)myrow >= (unsigned)P) report_internal(status);
         const uint4* src = x + t * H8;
-        for (int m0 = 0; m0 < nunits; m0 += 32 * U) {
-            uint4 q[U];
+        if (t + nw < T) {  // the warp's next token into L2 while this one is quantised
+            const char* nxt = reinterpret_cast<const char*>(x + (t + nw) * H8);
+            for (long long o = (long long)lane * 128; o < H * 2; o += 32 * 128)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(nxt + o));
+        }
+        for (int m0 = 0; m0 < nunits; m0 += 32 * L) {
+            uint4 a[L], b[L];
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int m = m0 + u * 32 + lane;
-                uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
+            for (int l = 0; l < L; ++l) {
+                const int m = m0 + l * 32 + lane;
+                a[l] = make_uint4(0, 0, 0, 0);
+                b[l] = make_uint4(0, 0, 0, 0);
                 if (m < nunits) {
-                    a = ld_stream_v4(src + 2 * m);
-                    b = ld_stream_v4(src + 2 * m + 1);
+                    a[l] = ld_stream_v4(src + 2 * m);
+                    b[l] = ld_stream_v4(src + 2 * m + 1);
                 }
-                const float f[16] = {bf16_lo(a.x), bf16_hi(a.x), bf16_lo(a.y), bf16_hi(a.y),
-                                     bf16_lo(a.z), bf16_hi(a.z), bf16_lo(a.w), bf16_hi(a.w),
-                                     bf16_lo(b.x), bf16_hi(b.x), bf16_lo(b.y), bf16_hi(b.y),
-                                     bf16_lo(b.z), bf16_hi(b.z), bf16_lo(b.w), bf16_hi(b.w)};
-                float amax = 0.0f;
-#pragma unroll
-                for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
-#pragma unroll
-                for (int o = 4; o >= 1; o >>= 1)
-                    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-                float sc;
-                if (amax == 0.0f) {
-                    sc = 1.0f;
-                    q[u] = make_uint4(0, 0, 0, 0);
-                } else {
-                    sc = __fdiv_rn(amax, 448.0f);
-                    const float inv = __fdiv_rn(448.0f, amax);
-                    float g[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) g[i] = __fmul_rn(f[i], inv);
-                    q[u].x = e4m3x2(g[0], g[1]) | (e4m3x2(g[2], g[3]) << 16);
-                    q[u].y = e4m3x2(g[4], g[5]) | (e4m3x2(g[6], g[7]) << 16);
-                    q[u].z = e4m3x2(g[8], g[9]) | (e4m3x2(g[10], g[11]) << 16);
-                    q[u].w = e4m3x2(g[12], g[13]) | (e4m3x2(g[14], g[15]) << 16);
-                }
-                if ((lane & 7) == 0 && m < nunits) wsc[m >> 3] = sc;
             }
-            for (int k = 0; k < K; ++k) {
-                const long long row = __shfl_sync(0xffffffffu, myrow, k);
-                if ((unsigned long long)row >= (unsigned long long)P) continue;  // range guard (reported above)
-                uint8_t* dst = recv + row * H;
 #pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const int m = m0 + u * 32 + lane;
-                    if (m < nunits) st_stream_v4(dst + (long long)m * 16, q[u]);
+            for (int g0 = 0; g0 < L; g0 += G) {
+                uint4 q[G];
+#pragma unroll
+                for (int u = 0; u < G; ++u) {
+                    const int l = g0 + u;
+                    const int m = m0 + l * 32 + lane;
+                    const float f[16] = {bf16_lo(a[l].x), bf16_hi(a[l].x), bf16_lo(a[l].y),
+                                         bf16_hi(a[l].y), bf16_lo(a[l].z), bf16_hi(a[l].z),
+                                         bf16_lo(a[l].w), bf16_hi(a[l].w), bf16_lo(b[l].x),
+                                         bf16_hi(b[l].x), bf16_lo(b[l].y), bf16_hi(b[l].y),
+                                         bf16_lo(b[l].z), bf16_hi(b[l].z), bf16_lo(b[l].w),
+                                         bf16_hi(b[l].w)};
+                    float amax = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+                    for (int o = 4; o >= 1; o >>= 1)
+                        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+                    float sc;
+                    if (amax == 0.0f) {
+                        sc = 1.0f;
+                        q[u] = make_uint4(0, 0, 0, 0);
+                    } else {
+                        sc = __fdiv_rn(amax, 448.0f);
+                        const float inv = __fdiv_rn(448.0f, amax);
+                        float g[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) g[i] = __fmul_rn(f[i], inv);
+                        q[u].x = e4m3x2(g[0], g[1]) | (e4m3x2(g[2], g[3]) << 16);
+                        q[u].y = e4m3x2(g[4], g[5]) | (e4m3x2(g[6], g[7]) << 16);
+                        q[u].z = e4m3x2(g[8], g[9]) | (e4m3x2(g[10], g[11]) << 16);
+                        q[u].w = e4m3x2(g[12], g[13]) | (e4m3x2(g[14], g[15]) << 16);
+                    }
+                    if ((lane & 7) == 0 && m < nunits) wsc[m >> 3] = sc;
+                }
+                for (int k = 0; k < K; ++k) {
+                    const long long row = __shfl_sync(0xffffffffu, myrow, k);
+                    if ((unsigned long long)row >= (unsigned long long)P) continue;  // range guard (reported above)
+                    uint8_t* dst = recv + row * H;
+#pragma unroll
+                    for (int u = 0; u < G; ++u) {
+                        const int m = m0 + (g0 + u) * 32 + lane;
+                        if (m < nunits) st_stream_v4(dst + (long long)m * 16, q[u]);
+                    }
                 }
             }
         }
@@ -155,6 +176,20 @@ int grid_for(long long work_warps, int blocks_per_sm) {
     if (want > cap) want = cap;
     if (want < 1) want = 1;
     return (int)want;
+}
+
+template <int L, int G>
+cudaError_t launch_fp8(const void* x, void* recv, float* recv_scale, const moonep_plan_t& p,
+                       const moonep_config& c, int grid, size_t smem, cudaStream_t s) {
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(dispatch_fp8_kernel<L, G>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    dispatch_fp8_kernel<L, G><<<grid, THREADS, smem, s>>>((const uint4*)x, (uint8_t*)recv,
+                                                          recv_scale, p.dst_row, p.status,
+                                                          c.R * c.S, c.K, c.H / 8);
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -180,30 +215,20 @@ cudaError_t launch_dispatch(const moonep_config& c, const moonep_plan_t& p, cons
             dispatch_bf16_kernel<2><<<grid, THREADS, 0, s>>>(
                 (const uint4*)x, (uint4*)recv, p.dst_row, p.status, T, c.K, H8);
     } else {
-        // four units (64 elements, 8 loads) per lane when the row has at least
-        // 2048 elements, and one warp per token (the grid covers every token,
-        // up to 256 blocks per SM, so the block scheduler balances the load):
-        // 0.956 of the copy peak at H = 4096, against 0.926 for two units on
-        // 32 blocks per SM and 0.84 for 8 elements per lane with 8-byte stores
-        const int grid = grid_for(T, 256);
+        // a whole 4096-element row (8 units, 16 loads) per lane and chunk when
+        // the row is that long, processed 4 units at a time, with the warp's
+        // next token requested into L2, on a grid of up to 128 blocks per SM
+        // (about 3 tokens per warp at the fp8 workload, so the request has
+        // time to land): 0.985 of the copy peak at H = 4096 (0.979-0.993 on
+        // grids of 64-128 blocks per SM), against 0.936-0.948 for four units
+        // per lane with one warp per token, on the same boxes, bit-identical
+        const int grid = grid_for(T, 128);
         const size_t smem = (size_t)WARPS * (H8 / 16) * sizeof(float);
-        if (H8 >= 256) {
-            if (smem > 48 * 1024) {
-                cudaError_t e = cudaFuncSetAttribute(
-                    dispatch_fp8_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-                if (e != cudaSuccess) return e;
-            }
-            dispatch_fp8_kernel<4><<<grid, THREADS, smem, s>>>(
-                (const uint4*)x, (uint8_t*)recv, recv_scale, p.dst_row, p.status, T, c.K, H8);
-        } else {
-            if (smem > 48 * 1024) {
-                cudaError_t e = cudaFuncSetAttribute(
-                    dispatch_fp8_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-                if (e != cudaSuccess) return e;
-            }
-            dispatch_fp8_kernel<2><<<grid, THREADS, smem, s>>>(
-                (const uint4*)x, (uint8_t*)recv, recv_scale, p.dst_row, p.status, T, c.K, H8);
-        }
+        if (H8 >= 512)
+            return launch_fp8<8, 4>(x, recv, recv_scale, p, c, grid, smem, s);
+        if (H8 >= 256)
+            return launch_fp8<4, 4>(x, recv, recv_scale, p, c, grid, smem, s);
+        return launch_fp8<2, 2>(x, recv, recv_scale, p, c, grid, smem, s);
     }
     return cudaGetLastError();
 }

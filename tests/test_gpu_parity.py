@@ -231,11 +231,13 @@ def test_determinism_zipf():
     assert torch.equal(ya.view(torch.int16), b["y"].view(torch.int16))
 
 
-@pytest.mark.parametrize("H", [128, 384, 1152, 4224])
+@pytest.mark.parametrize("H", [128, 384, 1152, 2176, 4224])
 def test_small_fp8_full(H):
     """fp8 payload element by element: codes, scales, dequantised expert and
     combine, over several hidden sizes (odd numbers of 128-blocks and of
-    32-lane passes), both rules, identity and scale experts."""
+    32-lane passes; each of the dispatch kernel's three shapes, and a row
+    longer than one 4096-element chunk), all rules, identity and scale
+    experts."""
     rng = np.random.default_rng(H)
     for it in range(6):
         cfgd = wl.random_small_cfg(rng, H=H)
