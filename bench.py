@@ -917,9 +917,11 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="moonep", choices=["moonep", "reference"])
-    ap.add_argument("--workload", default="hot",
-                    help="the step's workload (default: the largest single-GPU one, R32 S8192 "
-                         "E384 K8 H7168 with half of all picks on one expert)")
+    ap.add_argument("--workload", default=None,
+                    help="the step's workload (default: the largest single-GPU one, hot: R32 "
+                         "S8192 E384 K8 H7168 with half of all picks on one expert); with "
+                         "--gemm-only the GEMM's routing and sizes (default: the fp8 workload's "
+                         "sizes with a bf16 payload)")
     ap.add_argument("--no-sweep", action="store_true",
                     help="leave out the skew sweep and the other workloads' points")
     ap.add_argument("--alpha", type=float, default=None)
@@ -950,6 +952,10 @@ def main(argv=None):
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     from dispatch_moonep_plan_b200 import workloads as wl
+    gemm_base = args.workload or "fp8"
+    args.payload_fp8 = args.workload == "fp8"  # --gemm-only --workload fp8: the fp8 payload
+    if args.workload is None:
+        args.workload = "hot"
     cfgd = wl.WORKLOADS[args.workload]
     if args.S is not None:
         cfgd = wl.cfg_with(args.workload, S=args.S, name=cfgd["name"].replace(
@@ -958,7 +964,7 @@ def main(argv=None):
         run_reference(args, cfgd)
         return
     if args.gemm_only:
-        run_gemm_only(args)
+        run_gemm_only(args, gemm_base)
         return
     if args.side_only or args.backward_only:
         run_part_only(args, cfgd)
@@ -1042,7 +1048,7 @@ def run_part_only(args, cfgd):
     print(json.dumps(dict(backward=out)), flush=True)
 
 
-def run_gemm_only(args):
+def run_gemm_only(args, base):
     import torch
     from dispatch_moonep_plan_b200 import moonep as me
     from dispatch_moonep_plan_b200 import workloads as wl
@@ -1051,11 +1057,10 @@ def run_gemm_only(args):
     def flush():
         flush_w.zero_()
 
-    if args.workload == "fp8":
+    if base == "fp8" and args.payload_fp8:
         out = measure_gemm_fp8(me, wl, flush, 1, reps=args.steps, S=args.S, rule=args.rule)
         print(json.dumps(dict(expert_gemm_fp8=out)), flush=True)
         return
-    base = "fp8" if args.workload == "uniform" else args.workload  # the default: fp8's sizes
     out = measure_gemm(me, wl, flush, 1, reps=args.steps, S=args.S, rule=args.rule, base=base,
                        Hp=args.Hp)
     print(json.dumps(dict(expert_gemm=out)), flush=True)

@@ -12,10 +12,13 @@
 //
 //  - one persistent CTA per SM: warp 0 issues TMA loads, one thread of warp 1
 //    issues tcgen05.mma, warps 2-5 drain the accumulator (192 threads);
-//  - bf16 payload: tile 128 rows x BN columns (BN = 256 when H' allows, else
-//    128), k-block 64: A = 128 x 64 bf16 rows of the dispatched block
-//    (K-major), B = 64 x BN of the weight row (H' contiguous, MN-major), both
-//    128-byte swizzled in shared memory;
+//  - bf16 payload: tile 256 rows x 256 columns when H' % 256 == 0 (else 128
+//    x BN, BN = 256 or 128), k-block 64: A = two 128 x 64 bf16 blocks of the
+//    dispatched rows (K-major), B = 64 x 256 of the weight row (H'
+//    contiguous, MN-major), both 128-byte swizzled in shared memory; each B
+//    block feeds one MMA per 128-row half, so B crosses into shared memory
+//    once per 256 rows (the shared-memory traffic per MMA, TMA writes plus
+//    tensor-core reads, is what bounds a one-CTA tile);
 //  - fp8 payload: A never exists in bf16 outside the SM.  Warp 6 streams the
 //    e4m3 tiles into a ring of 4 slots, 8 converter warps widen them
 //    (a = bf16(float(q) * scale)) straight into tensor memory with
@@ -24,9 +27,10 @@
 //    N = 192, so A is widened once per 384 output columns (4 times per row
 //    block at H' = 1536, not 8).  One 384-column accumulator and 3 A stages
 //    (32 columns each) fit the 512 columns; the last n-tile may be partial;
-//  - the fp32 accumulator lives in tensor memory; the bf16 payload keeps two
-//    buffers of BN columns, so the epilogue of one tile overlaps the main
-//    loop of the next (the fp8 payload's single buffer does not);
+//  - the fp32 accumulator lives in tensor memory; with 128-row tiles there
+//    are two buffers, so the epilogue of one tile overlaps the main loop of
+//    the next (the 256 x 256 and the fp8 tiles fill the 512 columns with one
+//    buffer, and their epilogue does not);
 //  - the epilogue reads 32 lanes x 32 columns per tcgen05.ld, rounds once to
 //    bf16 (round-to-nearest-even) and stores only the rows of the group.
 //
@@ -238,7 +242,7 @@ struct GemmArgs {
     int debug_stall;  // epilogue waits on a barrier nothing completes
 };
 
-template <int BN, int STAGES, bool FP8A, int CW, int A8_SLOTS, int NSUB>
+template <int BN, int STAGES, bool FP8A, int CW, int A8_SLOTS, int NSUB, int MT>
 __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
     expert_gemm_kernel(const __grid_constant__ CUtensorMap tmX,
                        const __grid_constant__ CUtensorMap tmW, GemmArgs p) {
@@ -247,19 +251,25 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
     // k-step share one A block (fp8 payload: A is widened once per TN columns)
     constexpr int TN = NSUB * BN;
     constexpr int B_BYTES = BK * TN * 2;
+    // bf16 payload: a tile may also be MT m-tiles high (TM = MT * BM rows):
+    // every B block loaded then feeds MT MMAs, one per 128-row half, so the
+    // B operand crosses into shared memory once per TM rows
+    constexpr int TM = MT * BM;
+    static_assert(MT == 1 || !FP8A, "fp8 payload: one m-tile per tile");
     // a stage of the MMA ring: bf16 A (SW128, K-major) | B.  fp8 payload: A
     // lives in tensor memory, so a stage holds only B, and the e4m3 tiles
     // land in their own ring of A8_SLOTS after the stages.
-    constexpr int STAGE_A = FP8A ? 0 : A_BYTES;
+    constexpr int STAGE_A = FP8A ? 0 : MT * A_BYTES;
     constexpr int STAGE_BYTES = STAGE_A + B_BYTES;
     constexpr int A8S = FP8A ? A8_SLOTS : 0;
     // NACC accumulators of TN columns (two, so that the epilogue of one tile
     // overlaps the next tile's main loop, when they fit); fp8 payload: then A
     // stage s at columns ACOL + 32 s (128 rows x 64 bf16, two per column)
-    constexpr int NACC = (FP8A ? 2 * TN + 32 * STAGES : 2 * TN) <= 512 ? 2 : 1;
+    constexpr int NACC = (FP8A ? 2 * TN + 32 * STAGES : 2 * MT * TN) <= 512 ? 2 : 1;
     constexpr int ACOL = NACC * TN;
-    constexpr int TMEM_COLS = FP8A ? 512 : NACC * TN;
-    static_assert(NACC * TN + (FP8A ? 32 * STAGES : 0) <= 512 && TN <= 512,
+    constexpr int ACC_COLS = MT * TN;  // one accumulator: the MT halves side by side
+    constexpr int TMEM_COLS = FP8A ? 512 : NACC * ACC_COLS;
+    static_assert(NACC * ACC_COLS + (FP8A ? 32 * STAGES : 0) <= 512 && ACC_COLS <= 512,
                   "accumulators (and fp8 A stages) in the 512 tensor-memory columns");
     static_assert(!FP8A || (CW % 4 == 0 && CW <= 16), "whole converter warps per lane quarter");
     // k-block of A: 128 rows x 128 B; one k-step (16 elements) = 32 B along a row.
@@ -330,7 +340,7 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
         pair_rg(i, r, g);
         const int hi = __ldg(p.cu + r * G + g);
         const int lo = g ? __ldg(p.cu + r * G + g - 1) : 0;
-        const int c = (hi - lo + BM - 1) / BM;
+        const int c = (hi - lo + TM - 1) / TM;
         pre[i] = c;
         sum += c;
     }
@@ -388,7 +398,7 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
                 int pair, mt, nt, r, g;
                 locate(tile, pair, mt, nt);
                 pair_rg(pair, r, g);
-                const int row0 = r * p.C + (g ? __ldg(p.cu + r * G + g - 1) : 0) + mt * BM;
+                const int row0 = r * p.C + (g ? __ldg(p.cu + r * G + g - 1) : 0) + mt * TM;
                 const int wrow0 = (r * G + g) * p.H;
                 // 64-column boxes of B inside H' (all of them unless the
                 // last n-tile is partial; the rest of the stage is not read
@@ -405,8 +415,10 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
                     if constexpr (FP8A) {  // A comes from the e4m3 producer and the converters
                         mbar_expect_tx(&full[s], nbox * 8192);
                     } else {
-                        mbar_expect_tx(&full[s], A_BYTES + nbox * 8192);
-                        tma_load_2d(a, &tmX, &full[s], kb * BK, row0);
+                        mbar_expect_tx(&full[s], MT * A_BYTES + nbox * 8192);
+#pragma unroll
+                        for (int h = 0; h < MT; ++h)  // rows past the buffer are zero-filled
+                            tma_load_2d(a + h * A_BYTES, &tmX, &full[s], kb * BK, row0 + h * BM);
                     }
 #pragma unroll
                     for (int j = 0; j < TN / 64; ++j)
@@ -443,11 +455,15 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
             for (int tile = blockIdx.x; tile < total && !abort_flag; tile += gridDim.x) {
                 if (!mbar_wait(&tempty[acc], acc_ph ^ 1, p.wait_ns, &abort_flag)) break;
                 asm volatile("tcgen05.fence::after_thread_sync;");
-                const uint32_t d = tmem + acc * TN;
-                // sub-tiles wholly past H' (a partial last n-tile) are skipped
-                int nt_, pair_, mt_;
+                const uint32_t d = tmem + acc * ACC_COLS;
+                // sub-tiles wholly past H' (a partial last n-tile), and halves
+                // wholly past the group's rows, are skipped
+                int nt_, pair_, mt_, r_, g_;
                 locate(tile, pair_, mt_, nt_);
+                pair_rg(pair_, r_, g_);
                 const int nsub = min(NSUB, (p.Hp - nt_ * TN + BN - 1) / BN);
+                const int grows = __ldg(p.cu + r_ * G + g_) - (g_ ? __ldg(p.cu + r_ * G + g_ - 1) : 0);
+                const int nhalf = min(MT, (grows - mt_ * TM + BM - 1) / BM);
                 bool ok = true;
                 for (int kb = 0; kb < kblocks; ++kb) {
                     // the TMA loads landed; fp8: and the converter warps have
@@ -463,19 +479,24 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
 #pragma unroll
                     for (int ks = 0; ks < BK / 16; ++ks) {
 #pragma unroll
-                        for (int sub = 0; sub < NSUB; ++sub) {
-                            if (sub >= nsub) break;
-                            // sub-tile sub: columns sub*BN.. of the accumulator and
-                            // B chunks sub*BN/64.. of the stage
-                            const uint32_t bsub = b + sub * (BN / 64) * 8192;
-                            if constexpr (FP8A)
-                                mma_bf16_tmem_a(d + sub * BN, tmem + ACOL + s * 32 + ks * 8,
-                                                sdesc(bsub + ks * 2048, 8192, 1024), idesc,
-                                                (kb | ks) ? 1u : 0u);
-                            else
-                                mma_bf16(d + sub * BN, sdesc(a + ks * 32, 16, 1024),
-                                         sdesc(bsub + ks * 2048, 8192, 1024), idesc,
-                                         (kb | ks) ? 1u : 0u);
+                        for (int h = 0; h < MT; ++h) {
+                            if (h >= nhalf) break;
+#pragma unroll
+                            for (int sub = 0; sub < NSUB; ++sub) {
+                                if (sub >= nsub) break;
+                                // half h, sub-tile sub: columns h*TN + sub*BN.. of the
+                                // accumulator, A rows of half h, B chunks sub*BN/64..
+                                const uint32_t bsub = b + sub * (BN / 64) * 8192;
+                                if constexpr (FP8A)
+                                    mma_bf16_tmem_a(d + sub * BN, tmem + ACOL + s * 32 + ks * 8,
+                                                    sdesc(bsub + ks * 2048, 8192, 1024), idesc,
+                                                    (kb | ks) ? 1u : 0u);
+                                else
+                                    mma_bf16(d + h * TN + sub * BN,
+                                             sdesc(a + h * A_BYTES + ks * 32, 16, 1024),
+                                             sdesc(bsub + ks * 2048, 8192, 1024), idesc,
+                                             (kb | ks) ? 1u : 0u);
+                            }
                         }
                     }
                     any = true;
@@ -510,35 +531,39 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
             uint64_t* bar = p.debug_stall ? never : &tfull[acc];
             if (!mbar_wait(bar, acc_ph, p.wait_ns, &abort_flag)) break;
             asm volatile("tcgen05.fence::after_thread_sync;");
-            const int row_in = mt * BM + q * 32 + lane;
-            const bool valid = glo + row_in < ghi;
-            uint16_t* yrow = p.y + (size_t)(r * p.C + glo + row_in) * p.Hp + nt * TN;
-            const uint32_t tbase = tmem + acc * TN + ((uint32_t)(q * 32) << 16);
 #pragma unroll 1
-            for (int c0 = 0; c0 < TN; c0 += 32) {
-                if (nt * TN + c0 >= p.Hp) break;  // partial last n-tile (warp-uniform)
-                uint32_t v[32];
-                asm volatile(
-                    "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,"
-                    "%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,"
-                    "%31}, [%32];"
-                    : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
-                      "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]),
-                      "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]),
-                      "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
-                      "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]),
-                      "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-                    : "r"(tbase + c0));
-                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-                if (valid) {
+            for (int h = 0; h < MT; ++h) {
+                if (mt * TM + h * BM >= ghi - glo) break;  // half past the group (warp-uniform)
+                const int row_in = mt * TM + h * BM + q * 32 + lane;
+                const bool valid = glo + row_in < ghi;
+                uint16_t* yrow = p.y + (size_t)(r * p.C + glo + row_in) * p.Hp + nt * TN;
+                const uint32_t tbase = tmem + acc * ACC_COLS + h * TN + ((uint32_t)(q * 32) << 16);
+#pragma unroll 1
+                for (int c0 = 0; c0 < TN; c0 += 32) {
+                    if (nt * TN + c0 >= p.Hp) break;  // partial last n-tile (warp-uniform)
+                    uint32_t v[32];
+                    asm volatile(
+                        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,"
+                        "%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,"
+                        "%31}, [%32];"
+                        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+                          "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]),
+                          "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]),
+                          "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
+                          "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]),
+                          "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+                        : "r"(tbase + c0));
+                    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                    if (valid) {
 #pragma unroll
-                    for (int j = 0; j < 32; j += 8) {
-                        uint4 o;
-                        o.x = pack_bf16x2(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
-                        o.y = pack_bf16x2(__uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
-                        o.z = pack_bf16x2(__uint_as_float(v[j + 4]), __uint_as_float(v[j + 5]));
-                        o.w = pack_bf16x2(__uint_as_float(v[j + 6]), __uint_as_float(v[j + 7]));
-                        *reinterpret_cast<uint4*>(yrow + c0 + j) = o;
+                        for (int j = 0; j < 32; j += 8) {
+                            uint4 o;
+                            o.x = pack_bf16x2(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+                            o.y = pack_bf16x2(__uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+                            o.z = pack_bf16x2(__uint_as_float(v[j + 4]), __uint_as_float(v[j + 5]));
+                            o.w = pack_bf16x2(__uint_as_float(v[j + 6]), __uint_as_float(v[j + 7]));
+                            *reinterpret_cast<uint4*>(yrow + c0 + j) = o;
+                        }
                     }
                 }
             }
@@ -558,7 +583,7 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
                     int pair, mt, nt, r, g;
                     locate(tile, pair, mt, nt);
                     pair_rg(pair, r, g);
-                    const int row0 = r * p.C + (g ? __ldg(p.cu + r * G + g - 1) : 0) + mt * BM;
+                    const int row0 = r * p.C + (g ? __ldg(p.cu + r * G + g - 1) : 0) + mt * TM;
                     bool ok = true;
                     for (int kb = 0; kb < kblocks; ++kb) {
                         const int j8 = (int)(issued % A8S);
@@ -603,7 +628,7 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
                 locate(tile, pair, mt, nt);
                 pair_rg(pair, r, g);
                 const long long grow =
-                    (long long)r * p.C + (g ? __ldg(p.cu + r * G + g - 1) : 0) + mt * BM + row;
+                    (long long)r * p.C + (g ? __ldg(p.cu + r * G + g - 1) : 0) + mt * TM + row;
                 const bool live = grow < nrows;  // rows past the block are zero-filled
                 const float* srow = p.scale + (live ? grow * nsc : 0);
                 // the scale of the next 128 columns is loaded one group ahead
@@ -701,13 +726,13 @@ bool encode_2d(CUtensorMap* m, const void* base, CUtensorMapDataType type, uint6
 // alignment slack + stages + e4m3 ring + barriers (3 per stage, 2 per e4m3
 // slot, 2 + 2 accumulator, drain, never) + TMEM address + per-warp sums +
 // the m-tile prefix
-size_t smem_bytes(int bn, int stages, int npairs, bool fp8a, int a8_slots = 2) {
-    return 1024 + (size_t)stages * ((fp8a ? 0 : A_BYTES) + BK * bn * 2) +
+size_t smem_bytes(int bn, int stages, int npairs, bool fp8a, int a8_slots = 2, int mt = 1) {
+    return 1024 + (size_t)stages * ((fp8a ? 0 : mt * A_BYTES) + BK * bn * 2) +
            (fp8a ? a8_slots * A8_BYTES : 0) +
            (size_t)(3 * stages + 2 * a8_slots + 6) * 8 + 8 + 32 * 4 + (size_t)(npairs + 1) * 4;
 }
 
-template <int BN, int STAGES, bool FP8A, int CW = 8, int A8_SLOTS = 2, int NSUB = 1>
+template <int BN, int STAGES, bool FP8A, int CW = 8, int A8_SLOTS = 2, int NSUB = 1, int MT = 1>
 cudaError_t launch_variant(const CUtensorMap& x, const CUtensorMap& w, const GemmArgs& a,
                            size_t smem, int grid, cudaStream_t s) {
     static std::mutex mu;
@@ -718,13 +743,13 @@ cudaError_t launch_variant(const CUtensorMap& x, const CUtensorMap& w, const Gem
     {
         std::lock_guard<std::mutex> lock(mu);
         if (dev < 0 || dev >= 64 || set[dev] < smem) {
-            e = cudaFuncSetAttribute(expert_gemm_kernel<BN, STAGES, FP8A, CW, A8_SLOTS, NSUB>,
+            e = cudaFuncSetAttribute(expert_gemm_kernel<BN, STAGES, FP8A, CW, A8_SLOTS, NSUB, MT>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return e;
             if (dev >= 0 && dev < 64) set[dev] = smem;
         }
     }
-    expert_gemm_kernel<BN, STAGES, FP8A, CW, A8_SLOTS, NSUB>
+    expert_gemm_kernel<BN, STAGES, FP8A, CW, A8_SLOTS, NSUB, MT>
         <<<grid, threads_for<FP8A, CW>(), smem, s>>>(x, w, a);
     return cudaGetLastError();
 }
@@ -781,6 +806,13 @@ cudaError_t launch_expert_gemm(const moonep_config& c, const moonep_plan_t& p, c
         return launch_variant<192, FP8_STAGES, true, 8, FP8_A8, FP8_TN / 192>(
             tx, tw, a, smem_bytes(FP8_TN, FP8_STAGES, np, true, FP8_A8), grid, s);
     if (c.Hp % 256 == 0) {
+#ifndef GEMM_MT1
+        // 256 x 256 tiles (two m-tiles per B block), one accumulator
+        if (smem_bytes(256, 3, np, false, 2, 2) <= (size_t)SMEM_LIMIT)
+            return launch_variant<256, 3, false, 8, 2, 1, 2>(tx, tw, a,
+                                                            smem_bytes(256, 3, np, false, 2, 2),
+                                                            grid, s);
+#endif
         if (smem_bytes(256, 4, np, false) <= (size_t)SMEM_LIMIT)
             return launch_variant<256, 4, false>(tx, tw, a, smem_bytes(256, 4, np, false), grid, s);
         if (smem_bytes(256, 3, np, false) <= (size_t)SMEM_LIMIT)
