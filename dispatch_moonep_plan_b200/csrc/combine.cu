@@ -7,11 +7,18 @@
 // bf16 (nearest even) at the end.  The k order is fixed, so the result does
 // not depend on the launch shape.
 //
-// One warp per token.  Lane k < K holds dst_row[t,k] and w[t,k]; each lane
-// owns U 16-byte chunks of the row and accumulates 8 floats per chunk.  Up to
-// K = 8 a lane loads its chunks of all K rows before accumulating; above that,
-// the next pick's chunks are loaded while the current ones are accumulated.
+// Up to K = 8 with H a multiple of 512 (the workloads' rows): the K rows'
+// 512-element chunks are staged in shared memory by bulk copies (one
+// cp.async.bulk per row and chunk, completion on an mbarrier), two stages per
+// warp, so the next chunk is in flight while this one is summed.  Otherwise
+// one warp per token reads the rows with 16-byte loads: lane k < K holds
+// dst_row[t,k] and w[t,k]; each lane owns U 16-byte chunks of the row and
+// accumulates 8 floats per chunk; up to K = 8 it loads its chunks of all K
+// rows before accumulating, above that the next pick's chunks are loaded while
+// the current ones are accumulated.
 #include <cuda_bf16.h>
+
+#include <mutex>
 
 #include "internal.cuh"
 
@@ -349,6 +356,128 @@ __global__ void __launch_bounds__(THREADS) combine_bwd_seq_kernel(const uint4* _
     }
 }
 
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+// Combine with the rows staged by bulk copies.  Each of the block's 8 warps
+// owns two stages of KMAX x CH bf16 in shared memory; for each (token, chunk)
+// of its tokens (last to first, like the loads-first kernel), lane k < K
+// copies row k's chunk into the stage with one cp.async.bulk, whose completion
+// the stage's mbarrier counts in bytes; the following (token, chunk) is in
+// flight while this one is summed.  The same fma chain in k order and one
+// bf16 rounding: bit-identical to the kernels above.  Every wait is bounded;
+// one that runs out sets TIMEOUT, lets the other stage's copies land (bounded)
+// and stops the warp.
+template <int CH, int KMAX>
+__global__ void __launch_bounds__(THREADS, 1) combine_bulk_kernel(const uint16_t* __restrict__ eo,
+                                                                 const float* __restrict__ w,
+                                                                 const int32_t* __restrict__ dst_row,
+                                                                 uint4* __restrict__ y,
+                                                                 int32_t* status, int T, int K,
+                                                                 int H,
+                                                                 unsigned long long wait_ns) {
+    static_assert(CH % 256 == 0, "whole 16-byte vectors per lane");
+    if (!block_status_ok(status)) return;
+    extern __shared__ __align__(1024) uint8_t stage_mem[];
+    __shared__ __align__(8) uint64_t bars[WARPS][2];
+    constexpr int STAGE = KMAX * CH * 2;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint8_t* buf = stage_mem + warp * 2 * STAGE;
+    if (lane == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars[warp][0])));
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars[warp][1])));
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+    const int P = T * K;
+    const int nch = H / CH;
+    const long long nw = (long long)gridDim.x * WARPS;
+    const long long wid = (long long)blockIdx.x * WARPS + warp;
+    const long long nitems = (wid < T ? (T - 1 - wid) / nw + 1 : 0) * nch;
+    // item i: chunk i % nch of token T - 1 - (wid + (i / nch) * nw)
+    auto issue = [&](long long i, int st) {
+        const long long t = T - 1 - (wid + (i / nch) * nw);
+        const int c = (int)(i % nch);
+        int row = lane < K ? __ldg(dst_row + t * K + lane) : 0;
+        if (lane < K && (unsigned)row >= (unsigned)P) {  // range guard: report, read row 0
+            report_internal(status);
+            row = 0;
+        }
+        uint64_t* bar = &bars[warp][st];
+        if (lane == 0)
+            asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(
+                             smem_u32(bar)),
+                         "r"((uint32_t)(K * CH * 2))
+                         : "memory");
+        __syncwarp();
+        // the stage was read by generic loads; order them before the copy
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        if (lane < K) {
+            const uint16_t* src = eo + (long long)row * H + (long long)c * CH;
+            asm volatile(
+                "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, "
+                "[%3];" ::"r"(smem_u32(buf + st * STAGE + lane * CH * 2)),
+                "l"(src), "r"((uint32_t)(CH * 2)), "r"(smem_u32(bar))
+                : "memory");
+        }
+    };
+    auto wait_stage = [&](int st, uint32_t parity, unsigned long long limit) -> bool {
+        const unsigned long long t0 = globaltimer_ns();
+        for (int it = 1;; ++it) {
+            uint32_t done;
+            asm volatile(
+                "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; "
+                "selp.u32 %0, 1, 0, p; }"
+                : "=r"(done)
+                : "r"(smem_u32(&bars[warp][st])), "r"(parity)
+                : "memory");
+            if (done) return true;
+            if ((it & 63) == 0 && globaltimer_ns() - t0 > limit) return false;
+        }
+    };
+    uint32_t ph[2] = {0, 0};
+    if (nitems > 0) issue(0, 0);
+    for (long long i = 0; i < nitems; ++i) {
+        const int st = (int)(i & 1);
+        if (i + 1 < nitems) issue(i + 1, st ^ 1);
+        if (!wait_stage(st, ph[st], wait_ns)) {
+            if (lane == 0) atomicMax(status + ST_STATUS, MOONEP_STATUS_TIMEOUT);
+            if (i + 1 < nitems) wait_stage(st ^ 1, ph[st ^ 1], wait_ns);  // its copies land first
+            return;
+        }
+        ph[st] ^= 1;
+        const long long t = T - 1 - (wid + (i / nch) * nw);
+        const int c = (int)(i % nch);
+        const float myw = lane < K ? __ldg(w + t * K + lane) : 0.0f;
+        constexpr int V = CH / 256;  // 16-byte vectors per lane
+        float acc[8 * V];
+#pragma unroll
+        for (int j = 0; j < 8 * V; ++j) acc[j] = 0.0f;
+#pragma unroll
+        for (int k = 0; k < KMAX; ++k) {
+            if (k < K) {
+                const float wk = __shfl_sync(0xffffffffu, myw, k);
+                const uint4* rowv = reinterpret_cast<const uint4*>(buf + st * STAGE + k * CH * 2);
+#pragma unroll
+                for (int v = 0; v < V; ++v) accum<true>(acc + 8 * v, wk, rowv[v * 32 + lane]);
+            }
+        }
+        uint4* dst = y + (t * H + (long long)c * CH) / 8;
+#pragma unroll
+        for (int v = 0; v < V; ++v) {
+            uint4 o;
+            o.x = pack_bf16x2(acc[8 * v + 0], acc[8 * v + 1]);
+            o.y = pack_bf16x2(acc[8 * v + 2], acc[8 * v + 3]);
+            o.z = pack_bf16x2(acc[8 * v + 4], acc[8 * v + 5]);
+            o.w = pack_bf16x2(acc[8 * v + 6], acc[8 * v + 7]);
+            dst[v * 32 + lane] = o;
+        }
+        __syncwarp();  // the stage is read before it is refilled
+    }
+}
+
 int grid_4_per_sm(long long T) {
     const int sms = device_sm_count();
     long long grid = (T + WARPS - 1) / WARPS;
@@ -423,6 +552,36 @@ cudaError_t launch_combine(const moonep_config& c, const moonep_plan_t& p, const
                            const float* w, void* y, cudaStream_t s) {
     const int T = c.R * c.S;
     const int H8 = c.H / 8;
+    if (c.K <= 8 && c.H % 512 == 0) {
+        // rows staged by bulk copies, 512-element chunks, one block of 8 warps
+        // per SM (128 KiB of stages): measured at the hot-expert workload 4957
+        // us against 4966 us for the loads-first kernel, 1.057 of the copy
+        // peak, bit-identical; 256-element chunks on 1-3 blocks per SM
+        // measured 0.66-0.97
+        constexpr int CH = 512;
+        const size_t smem = (size_t)WARPS * 2 * 8 * CH * 2;
+        static std::mutex mu;
+        static bool set[64] = {};
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        {
+            std::lock_guard<std::mutex> lock(mu);
+            if (dev < 0 || dev >= 64 || !set[dev]) {
+                e = cudaFuncSetAttribute(combine_bulk_kernel<CH, 8>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+                if (e != cudaSuccess) return e;
+                if (dev >= 0 && dev < 64) set[dev] = true;
+            }
+        }
+        long long grid = device_sm_count();
+        if (grid > T) grid = T;
+        if (grid < 1) grid = 1;
+        combine_bulk_kernel<CH, 8><<<(int)grid, THREADS, smem, s>>>(
+            (const uint16_t*)eo, w, p.dst_row, (uint4*)y, p.status, T, c.K, c.H,
+            current_wait_limit_ns());
+        return cudaGetLastError();
+    }
     if (c.K <= 8) {
         combine_kfirst_kernel<2, 8, true><<<grid_warp_per_token(T), THREADS, 0, s>>>(
             (const uint4*)eo, w, p.dst_row, (uint4*)y, p.status, T, c.K, H8);

@@ -63,6 +63,24 @@ def test_many_picks_per_token(shape):
             _full_check(cfgd, idx, w, seed=seed, rule=rule, expert="scale")
 
 
+@pytest.mark.parametrize("shape", [
+    (2, 37, 8, 3, 4, 512),      # one 512-element chunk per row, ragged token count
+    (3, 50, 9, 8, 3, 1024),     # K = 8, two chunks
+    (1, 5, 4, 1, 0, 512),       # one rank, one pick per token, fewer tokens than warps
+    (4, 23, 8, 5, 3, 1536),     # three chunks, K = 5
+])
+def test_combine_bulk_staged(shape):
+    """Rows of a multiple of 512 elements with K <= 8 take the combine that
+    stages the rows in shared memory with bulk copies: every token against the
+    oracle, bit for bit, under all rules and the scale expert."""
+    R, S, E, K, B, H = shape
+    cfgd = _cfg(R, S, E, K, B, H, alpha=1.2)
+    for seed in range(2):
+        idx, w = wl.routing(cfgd, seed=seed)
+        for rule in (0, 1, 2):
+            _full_check(cfgd, idx, w, seed=seed, rule=rule, expert="scale")
+
+
 def test_largest_E_and_R():
     cfgd = _cfg(128, 16, 1024, 8, 16, 64, alpha=1.2)
     idx, w = wl.routing(cfgd, seed=0)
