@@ -7,7 +7,7 @@
 // bf16 (nearest even) at the end.  The k order is fixed, so the result does
 // not depend on the launch shape.
 //
-// Up to K = 8 with H a multiple of 512 (the workloads' rows): the K rows'
+// Up to K = 8 with H a multiple of 512 and at least 4096: the K rows'
 // 512-element chunks are staged in shared memory by bulk copies (one
 // cp.async.bulk per row and chunk, completion on an mbarrier), two stages per
 // warp, so the next chunk is in flight while this one is summed.  Otherwise
@@ -552,12 +552,13 @@ cudaError_t launch_combine(const moonep_config& c, const moonep_plan_t& p, const
                            const float* w, void* y, cudaStream_t s) {
     const int T = c.R * c.S;
     const int H8 = c.H / 8;
-    if (c.K <= 8 && c.H % 512 == 0) {
+    if (c.K <= 8 && c.H % 512 == 0 && c.H >= 4096) {
         // rows staged by bulk copies, 512-element chunks, one block of 8 warps
-        // per SM (128 KiB of stages): measured at the hot-expert workload 4957
-        // us against 4966 us for the loads-first kernel, 1.057 of the copy
-        // peak, bit-identical; 256-element chunks on 1-3 blocks per SM
-        // measured 0.66-0.97
+        // per SM (128 KiB of stages): 1.057-1.061 of the copy peak at H = 4096
+        // and 7168 (the loads-first kernel: 1.052-1.057), bit-identical; at
+        // H = 2048 (4 chunks a token, K = 6) 0.83 against 1.00, so shorter
+        // rows take the loads-first kernel; 256-element chunks on 1-3 blocks
+        // per SM measured 0.66-0.97
         constexpr int CH = 512;
         const size_t smem = (size_t)WARPS * 2 * 8 * CH * 2;
         static std::mutex mu;

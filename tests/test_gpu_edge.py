@@ -64,15 +64,16 @@ def test_many_picks_per_token(shape):
 
 
 @pytest.mark.parametrize("shape", [
-    (2, 37, 8, 3, 4, 512),      # one 512-element chunk per row, ragged token count
-    (3, 50, 9, 8, 3, 1024),     # K = 8, two chunks
-    (1, 5, 4, 1, 0, 512),       # one rank, one pick per token, fewer tokens than warps
-    (4, 23, 8, 5, 3, 1536),     # three chunks, K = 5
+    (2, 37, 8, 3, 4, 4096),     # 8 chunks of 512 per row, ragged token count
+    (3, 50, 9, 8, 3, 4608),     # K = 8, 9 chunks
+    (1, 5, 4, 1, 0, 4096),      # one rank, one pick per token, fewer tokens than warps
+    (4, 23, 8, 5, 3, 7168),     # the hot workload's row length, K = 5
 ])
 def test_combine_bulk_staged(shape):
-    """Rows of a multiple of 512 elements with K <= 8 take the combine that
-    stages the rows in shared memory with bulk copies: every token against the
-    oracle, bit for bit, under all rules and the scale expert."""
+    """Rows of at least 4096 elements (a multiple of 512) with K <= 8 take the
+    combine that stages the rows in shared memory with bulk copies: every
+    token against the oracle, bit for bit, under all rules and the scale
+    expert."""
     R, S, E, K, B, H = shape
     cfgd = _cfg(R, S, E, K, B, H, alpha=1.2)
     for seed in range(2):
