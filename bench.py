@@ -421,6 +421,9 @@ def run_gpu(args, cfgd, emit=True):
             m_graph, graph_note = graph_step_time(step, flush, args, world, stream)
     step_ms = m_graph if m_graph is not None else m_step
     clocks = clk_g.summary() if m_graph is not None else clk.summary()
+    # each kernel's interval inside one captured step, events as graph nodes
+    ig = graph_node_times(lambda ev, st: step(ev, st), 5, flush, args, stream)
+    ig = reduce_max(ig if ig else [float("nan")] * 4, world)
 
     # ---- end to end through the C ABI with host buffers ----
     if getattr(args, "no_e2e", False):
@@ -446,6 +449,11 @@ def run_gpu(args, cfgd, emit=True):
                       frac=dom_gbs / peak, traffic=traffic,
                       algorithmic_bytes=bytes_[dom], peak_kind=peak_kind),
         plan_us=m_plan * 1e3, dispatch_us=m_disp * 1e3, combine_us=m_comb * 1e3,
+        in_graph=dict(plan_us=ig[0], dispatch_us=ig[1], combine_us=ig[3],
+                      how="the step captured once as a CUDA graph with its events as graph "
+                          "nodes between the kernels; median of the K replays (L2 flushed "
+                          "before each); the keys above time each kernel by events on the "
+                          "stream around its own launch"),
         dispatch_GBps=disp_gbs, combine_GBps=comb_gbs,
         dispatch_frac=disp_gbs / peak, combine_frac=comb_gbs / peak,
         maxvio=maxvio, tokens_per_s=world * T / (step_ms * 1e-3),
@@ -472,6 +480,37 @@ def run_gpu(args, cfgd, emit=True):
         import torch.distributed as dist
         dist.destroy_process_group()
     return out if rank == 0 else None
+
+
+def graph_node_times(body, n_events, flush, args, stream):
+    """Capture body(events, stream) once as a CUDA graph whose events are
+    graph nodes, replay it W + K times (L2 flushed before each, outside the
+    graph) and return the median of each interval between consecutive events
+    over the K timed replays, in µs; None if the capture is not supported."""
+    import torch
+    try:
+        ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_events)]
+        cs = torch.cuda.Stream()
+        cs.wait_stream(stream)
+        with torch.cuda.stream(cs):
+            body(ev, cs)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cs):
+            body(ev, cs)
+        torch.cuda.synchronize()
+    except Exception:
+        return None
+    iv = [[] for _ in range(n_events - 1)]
+    for i in range(args.warmup + args.steps):
+        flush()
+        g.replay()
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            for j in range(n_events - 1):
+                iv[j].append(ev[j].elapsed_time(ev[j + 1]) * 1e3)
+    del g
+    return [statistics.median(v) for v in iv]
 
 
 def graph_step_time(step, flush, args, world, stream):
@@ -1010,10 +1049,16 @@ def run_plan_only(args, cfgd):
         b.record(stream)
         torch.cuda.synchronize()
         ts.append(a.elapsed_time(b) * 1e3)
+    # the same call as a node of a CUDA graph, events recorded as graph nodes
+    # on both sides (how the planner runs inside the captured step)
+    tg = graph_node_times(lambda ev, st: (ev[0].record(st), me.plan(cfg, idx_d, bufs, st),
+                                          ev[1].record(st)),
+                          2, flush_w.zero_, args, stream)
     print(json.dumps(dict(plan=dict(workload=cfgd["name"], rule=args.rule, status=st,
                                     maxvio=float(bufs.maxvio.item()),
                                     plan_us=statistics.median(ts), mean_us=statistics.mean(ts),
-                                    min_us=min(ts), calls=len(ts)))), flush=True)
+                                    min_us=min(ts), calls=len(ts),
+                                    plan_us_in_graph=tg[0] if tg else None))), flush=True)
 
 
 def run_part_only(args, cfgd):

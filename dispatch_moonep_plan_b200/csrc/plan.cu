@@ -12,29 +12,34 @@
 // Kernel structure (one block per SM, 1024 threads, cooperative launch so
 // that every block is resident and the grid-wide wait cannot deadlock):
 //   A. each block owns a contiguous run of picks, each warp a contiguous part
-//      of it; every warp takes its picks 32 at a time in (t, k) order, finds
-//      the lanes holding the same expert (match.any), and the lowest of them
-//      adds their number to the warp's shared histogram; the count it finds
-//      there (the expert's picks in the warp's earlier rows) plus the lane's
-//      rank among them is the pick's position among the warp's picks of that
-//      expert, kept beside the pick in shared memory; the block writes its
-//      row hist[block][e].
-//   -- one grid-wide wait --
+//      of it; every warp ranks its picks 32 at a time in (t, k) order: the
+//      lanes holding the same expert are found (one ballot for lane 0's
+//      expert, lane-mask words in shared memory for the rest, or match.any
+//      when the words do not fit), and the group's lowest lane advances the
+//      warp's count of that expert; count before the row plus the lane's rank
+//      in its group is the pick's position among the warp's picks of the
+//      expert, kept beside the pick in shared memory.  One warp per expert
+//      then scans the 32 warps' counts: the block's row hist[block][e] and
+//      each warp's offset within the block.
+//   -- one grid-wide wait; while it lasts, each block sorts its own picks
+//      into expert-major order in shared memory (slot = the block's prefix
+//      over experts + the warp's offset + the position in the warp) --
 //   B. every block reads all rows of hist (16-byte loads when E % 4 == 0):
 //      the per-expert totals, and the counts of the blocks before it (its
 //      offsets).
 //   C. every block computes the small O(E + R) balance step itself from the
 //      totals (no further grid-wide wait is needed); block 0 writes the
 //      per-layer outputs, each block writes cu_seqlens / slot_expert of the
-//      ranks it owns; then every warp walks its picks again: a pick's position
-//      among all picks of its expert is the block's offset plus the counts of
-//      the block's earlier warps plus its position within the warp, so the
-//      placement is stable and deterministic without ordered atomics, and the
-//      picks of a row are placed independently.  The destination comes from
-//      one 16-byte per-expert table entry (kept rows) or a short search of
-//      the receiving segments (overflow rows).  When a block's picks do not
-//      fit in shared memory, the walk reads them again and recomputes the
-//      positions row by row with running per-warp offsets.
+//      ranks it owns; then the block places its picks in expert-major order:
+//      slot i of expert e is the pick at position i + offset(e) among all
+//      picks of e, so the placement is stable and deterministic without
+//      ordered atomics.  Its row comes from one 16-byte per-expert table
+//      entry (kept rows) or, for overflow, a bucket table over the overflow
+//      stream.  Consecutive threads write consecutive rows of the inverse map;
+//      the forward map is collected in shared memory and written out in pick
+//      order.  When a block's picks do not fit in shared memory, the walk
+//      reads them again in (t, k) order and ranks them row by row against
+//      running per-warp offsets.
 // The wait is bounded (globaltimer); when it runs out the block records
 // MOONEP_STATUS_TIMEOUT and returns.
 #include <algorithm>
@@ -49,6 +54,7 @@ constexpr int NW = THREADS / 32;
 constexpr int UNR = 8;   // picks per lane loaded ahead in the streaming loops
 constexpr int BUNR = 8;  // histogram rows per thread loaded ahead in phase B
 constexpr int SCAN_N = 4;
+constexpr int NBKT = 512;  // buckets of the overflow stream (receiving-position lookup)
 
 struct PlanParams {
     int R, S, E, K, B, rule, Er, C, P;
@@ -69,11 +75,20 @@ struct PlanParams {
 };
 
 struct Smem {
-    int* whist;   // [NW][E] per-warp counts, later per-warp running offsets
+    int* whist;   // [NW][WS] per-warp counts; then each warp's offset among the
+                  //          block's picks of the expert, plus the expert's
+                  //          first expert-major slot (picks kept) or the
+                  //          block's offset among all its picks (not kept)
+    unsigned* wmask;  // [NW][WS] per-warp lane masks of the row being ranked
+                      //          (ranking by masks only); shares its space with
+    int* sorted;  // [chunk] the block's picks in expert-major order: expert |
+                  //         (pick - first pick of the block) << 10 (kept picks)
     int* cnt;     // [E]   picks of each expert (all blocks)
     int* bcnt;    // [E]   picks of each expert in this block
     int* bpre;    // [E]   picks of each expert in the blocks before this one
     int* kk;      // [E]   rows of each expert kept on its home rank
+    int* nzlist;  // [E]   experts with overflow, in stream order
+    int* bex;     // [E]   exclusive prefix of bcnt over experts (expert-major slots)
     int* pc;      // [E+1] exclusive prefix of cnt over experts
     int* pk;      // [E+1] exclusive prefix of kk over experts
     int* ov;      // [E]   rows of each expert that overflow its home rank
@@ -81,11 +96,12 @@ struct Smem {
     int* osi;     // [E+1] start of the stream item at each position (non-decreasing)
     int* nzri;    // [E+1] items with overflow before each position
     int* ose;     // [E]   start of each expert's rows in the overflow stream
-    int* nzlist;  // [E]   experts with overflow, in stream order
     int4* tab;    // [E]   per expert: rows kept, destination row of its first kept
-                  //       pick, overflow-stream index of pick 0 (ose - kept), picks
-    int* rng;     // [E]   positions of the receiving order that take the expert's
-                  //       overflow: first | last << 16
+                  //       pick, overflow-stream index of pick 0 (ose - kept), picks;
+                  //       on the expert-major path shifted to index by slot
+    int* bkt;     // [NBKT] per bucket of 2^sh consecutive overflow-stream indices:
+                  //       the receiving positions of its first and last index,
+                  //       first | last << 16
     int* kept;    // [R]
     int* def;     // [R] C - kept
     int* segs;    // [R] start of the rank's segment in the stream
@@ -97,32 +113,46 @@ struct Smem {
     int* sege_at; // [R] segment end at each position of the receiving order
     int* rbase;   // [R] destination row of stream index 0 at each receiving position
     int* scratch; // [2*SCAN_N*32 + 8]
-    int* stash;   // [chunk] the block's picks (when stashed)
+    int* stash;   // [chunk] the block's picks in (t, k) order, expert | position
+                  //         in the warp << 10; later each pick's destination row
 };
 
-__host__ __device__ inline size_t smem_ints(int E, int R) {
-    return (size_t)NW * E + 13 * (size_t)E + 3 + 4 * ((size_t)E + 1) + 10 * (size_t)R +
-           2 * SCAN_N * 32 + 8;
+// Row stride of the per-warp arrays: odd, so that the 32 warps' entries of
+// one expert lie in 32 different banks.
+__host__ __device__ inline int warp_stride(int E) { return E | 1; }
+
+__host__ __device__ inline size_t smem_ints(int E, int R, bool mask, bool stash, long long chunk) {
+    const size_t nw = (size_t)NW * warp_stride(E);
+    const size_t c = stash ? (size_t)chunk : 0;
+    const size_t u = mask ? (nw > c ? nw : c) : c;  // wmask and sorted share
+    return (size_t)((E + 3) & ~3) + 4 * (size_t)E + nw + u + 6 * (size_t)E +
+           4 * ((size_t)E + 1) + 2 * (size_t)E + NBKT + 10 * (size_t)R + 2 * SCAN_N * 32 + 8 + c;
 }
 
-__device__ inline Smem carve(int* base, int E, int R) {
+__device__ inline Smem carve(int* base, int E, int R, bool mask, bool stash, int chunk) {
     Smem s;
     int* p = base;
     s.ov = p; p += (E + 3) & ~3;  // first and padded: read four at a time
     s.tab = reinterpret_cast<int4*>(p); p += 4 * E;  // 16-byte aligned after ov
-    s.whist = p; p += NW * E;
+    const int nw = NW * warp_stride(E);
+    const int c = stash ? chunk : 0;
+    s.whist = p; p += nw;
+    s.wmask = reinterpret_cast<unsigned*>(p);
+    s.sorted = p;
+    p += mask ? (nw > c ? nw : c) : c;
     s.cnt = p; p += E;
     s.bcnt = p; p += E;
     s.bpre = p; p += E;
     s.kk = p; p += E;
     s.nzlist = p; p += E;
+    s.bex = p; p += E;
     s.pc = p; p += E + 1;
     s.pk = p; p += E + 1;
     s.item_at = p; p += E;
     s.osi = p; p += E + 1;
     s.nzri = p; p += E + 1;
     s.ose = p; p += E;
-    s.rng = p; p += E;
+    s.bkt = p; p += NBKT;
     s.kept = p; p += R;
     s.def = p; p += R;
     s.segs = p; p += R;
@@ -187,21 +217,30 @@ __device__ __forceinline__ int upper_bound(const int* a, int n, int v) {
     return lo;
 }
 
-// Grid-wide wait with a time limit.  Returns false if it ran out.
+// Grid-wide barrier, in two halves so that a block can work on its own data
+// between them.  Arrive (after the block's __syncthreads, which orders the
+// block's writes before thread 0's next operation): thread 0 counts the block
+// in with a release add at gpu scope, which makes those writes visible to
+// every thread that acquires the count.
+__device__ __forceinline__ void grid_arrive(unsigned* ctr) {
+    if (threadIdx.x == 0) red_release_add_u32(ctr, 1u);
+}
+
+// Wait, with a time limit, until target blocks have arrived.  Returns false
+// if it ran out.
 __device__ bool grid_wait(unsigned* ctr, unsigned target, unsigned long long limit_ns, int* flag) {
     __syncthreads();
     if (threadIdx.x == 0) {
-        __threadfence();
-        red_release_add_u32(ctr, 1u);
         const unsigned long long t0 = globaltimer_ns();
         int ok = 1;
+        // acquire loads: the other blocks' writes before their arrival are
+        // visible to thread 0, and to the block after the barrier below
         while (ld_acquire_u32(ctr) < target) {
             if (globaltimer_ns() - t0 > limit_ns) {
                 ok = 0;
                 break;
             }
         }
-        __threadfence();
         *flag = ok;
     }
     __syncthreads();
@@ -220,7 +259,10 @@ __device__ int balance(const PlanParams& p, Smem& s, int* misc) {
 
     // q = rows of the same rank's experts that are kept before expert e
     int q = 0;
-    if (p.rule == MOONEP_RULE_INDEX_ORDER) {
+    if (p.rule == MOONEP_RULE_INDEX_ORDER && Er <= 32) {
+        if (ve)
+            for (int i = first; i < e; ++i) q += s.cnt[i];  // at most 31 loads
+    } else if (p.rule == MOONEP_RULE_INDEX_ORDER) {
         int v1[1] = {c}, ex1[1], t1[1];
         block_scan<1>(v1, ex1, t1, s.scratch);
         if (ve) s.pc[e] = ex1[0];
@@ -362,15 +404,20 @@ __device__ int balance(const PlanParams& p, Smem& s, int* misc) {
     return misc[0] >= 0 ? MOONEP_STATUS_SLOT_BUDGET : MOONEP_STATUS_OK;
 }
 
-// Destination row of the pick at position pos among expert e's picks (t =
+// Destination row of the pick at position pos among its expert's picks (t =
 // the expert's table entry), or -1 if its stream index is past every segment.
-__device__ __forceinline__ int place(const PlanParams& p, const Smem& s, int e, const int4& t,
-                                     int pos) {
+// An overflow pick's receiving position is the first whose segment ends past
+// its stream index; the bucket of 2^sh indices holding it gives the positions
+// of the bucket's first and last index, between which the answer lies (almost
+// always one and the same).
+__device__ __forceinline__ int place(const PlanParams& p, const Smem& s, const int4& t, int pos,
+                                     int sh) {
     if (pos < t.x) return t.y + pos;  // kept on the home rank
     const int sidx = t.z + pos;       // index in the overflow stream
-    // the receiving position lies in [first, last] of the receiving order
-    const int rr = s.rng[e];
-    int lo = rr & 0xffff, hi = (rr >> 16) + 1;
+    const int bi = sidx >> sh;
+    if (sidx < 0 || bi >= NBKT) return -1;
+    const int bb = s.bkt[bi];
+    int lo = bb & 0xffff, hi = bb >> 16;
     while (lo < hi) {
         const int mid = (lo + hi) >> 1;
         if (s.sege_at[mid] <= sidx) lo = mid + 1;
@@ -385,23 +432,80 @@ __device__ __forceinline__ int place(const PlanParams& p, const Smem& s, int e, 
 // < 2^31 / (148 * 32) + 1 picks).
 __device__ __forceinline__ int pack_pick(int e, int off) { return e | (off << 10); }
 
+// Stable ranking of one row (32 consecutive picks, one per lane; e = -1 for
+// none) within a warp: returns the lane's position among the warp's picks of
+// its expert so far (the counts in wh from earlier rows, then the row's lower
+// lanes holding the same expert) and moves wh[e] past the row.
+//   MASK: the lanes holding the warp's candidate expert are found by one
+//   ballot; every other lane ORs its bit into its expert's mask word wm[e],
+//   and after the warp's barrier one read gives the whole group, so the rank
+//   does not depend on the order the atomics were carried out in.  The
+//   candidate (warp-uniform) stays while it holds 4 or more lanes of a row,
+//   else it becomes the expert of the lowest lane outside it: under a heavy
+//   skew it settles on the hot expert, whose lanes would otherwise all set
+//   bits in one word, one after another.
+//   The group's lowest lane advances the count and clears the word (every
+//   word is zero between rows).  Top-k routing keeps the lanes sharing a word
+//   few: a token's k experts are distinct, so at most ceil(31 / k) + 1 lanes
+//   of a row hold one expert.
+//   Otherwise match.any finds the group (its cost grows with the number of
+//   distinct experts in the row, about ten times the masks' at 30).
+template <bool MASK>
+__device__ __forceinline__ int rank_row(int* wh, unsigned* wm, int e, int lane, unsigned lt_mask,
+                                        int& cand) {
+    unsigned m;
+    if constexpr (MASK) {
+        const unsigned mc = __ballot_sync(0xffffffffu, e >= 0 && e == cand);
+        const bool inc = (mc >> lane) & 1u;
+        if (e >= 0 && !inc) atomicOr(wm + e, 1u << lane);
+        if (__popc(mc) < 4) {
+            const unsigned rest = __ballot_sync(0xffffffffu, e >= 0) & ~mc;
+            if (rest) cand = __shfl_sync(0xffffffffu, e, __ffs(rest) - 1);
+        }
+        __syncwarp();
+        m = inc ? mc : (e >= 0 ? wm[e] : 0u);
+    } else {
+        m = __match_any_sync(0xffffffffu, e);
+    }
+    const int run = e >= 0 ? wh[e] : 0;
+    __syncwarp();
+    const int rank = __popc(m & lt_mask);
+    if (e >= 0 && rank == 0) {
+        wh[e] = run + __popc(m);
+        if constexpr (MASK) wm[e] = 0u;
+    }
+    __syncwarp();
+    return run + rank;
+}
+
+template <bool MASK>
 __global__ void __launch_bounds__(THREADS, 1) plan_kernel(PlanParams p) {
     extern __shared__ __align__(16) int smem_raw[];
-    Smem s = carve(smem_raw, p.E, p.R);
+    const bool stash = p.stash != 0;
+    Smem s = carve(smem_raw, p.E, p.R, MASK, stash, p.chunk);
     __shared__ int wait_flag;
     __shared__ int max_count;
     __shared__ int misc[4];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int G = gridDim.x, b = blockIdx.x;
-    const int E = p.E;
+    const int E = p.E, WS = warp_stride(E);
     const long long P = p.P;
-    const long long clo = P * b / G, chi = P * (b + 1) / G, len = chi - clo;
-    const long long wlo = clo + len * warp / NW, whi = clo + len * (warp + 1) / NW;
-    int* wh = s.whist + warp * E;
+    // pick indices in 32 bits: P < 2^31, so even a row's last lane (< P + 256)
+    // fits without wrapping
+    const unsigned clo = (unsigned)(P * b / G), chi = (unsigned)(P * (b + 1) / G);
+    const int len = (int)(chi - clo);
+    const unsigned wlo = clo + (unsigned)((long long)len * warp / NW);
+    const unsigned whi = clo + (unsigned)((long long)len * (warp + 1) / NW);
+    int* wh = s.whist + warp * WS;
+    unsigned* wm = s.wmask + warp * WS;  // used only when MASK
+    const unsigned lt_mask = (1u << lane) - 1u;
 
-    // ---- A: per-warp histograms ----------------------------------------
-    for (int i = tid; i < NW * E; i += THREADS) s.whist[i] = 0;
+    // ---- A: per-warp histograms and positions within the warp ---------------
+    for (int i = tid; i < NW * WS; i += THREADS) {
+        s.whist[i] = 0;
+        if constexpr (MASK) s.wmask[i] = 0u;
+    }
     for (int i = tid; i < E; i += THREADS) {
         s.cnt[i] = 0;
         s.bpre[i] = 0;
@@ -409,48 +513,89 @@ __global__ void __launch_bounds__(THREADS, 1) plan_kernel(PlanParams p) {
     if (tid == 0) max_count = 0;
     __syncthreads();
     int bad = 0;
-    const unsigned lt_mask = (1u << lane) - 1u;
-    for (long long base = wlo; base < whi; base += 32 * UNR) {
+    int cand = -1;  // the warp's candidate expert (ranking by masks)
+    for (unsigned base = wlo; base < whi; base += 32 * UNR) {
         int ev[UNR];
 #pragma unroll
         for (int u = 0; u < UNR; ++u) {
-            const long long q = base + u * 32 + lane;
+            const unsigned q = base + u * 32 + lane;
             ev[u] = q < whi ? __ldg(p.idx + q) : -1;
         }
 #pragma unroll
         for (int u = 0; u < UNR; ++u) {
             if (base + u * 32 < whi) {  // warp-uniform: the row has picks
-                const long long q = base + u * 32 + lane;
+                const unsigned q = base + u * 32 + lane;
                 const bool valid = q < whi;
                 const int e = ev[u];
                 const bool ok = valid && e >= 0 && e < E;
                 if (valid && !ok) bad = 1;
-                // lanes of the row holding the same expert; every other lane
-                // (no pick, or a bad index) shares the key -1
-                const unsigned peers = __match_any_sync(0xffffffffu, ok ? e : -1);
-                const int rank = __popc(peers & lt_mask);
-                // the lowest lane adds the group's picks; the count it found
-                // is the group's position in the warp's picks of the expert.
-                // The next row's adds come after this one (shuffle, then the
-                // warp's memory-ordering barrier).
-                const int before = (ok && rank == 0) ? atomicAdd(wh + e, __popc(peers)) : 0;
-                const int off = __shfl_sync(0xffffffffu, before, __ffs(peers) - 1) + rank;
-                __syncwarp();
-                if (ok && p.stash) s.stash[q - clo] = pack_pick(e, off);
+                // a lane with no pick, or a bad index, takes no part
+                const int off = rank_row<MASK>(wh, wm, ok ? e : -1, lane, lt_mask, cand);
+                if (valid && stash) s.stash[q - clo] = ok ? pack_pick(e, off) : -1;
             }
         }
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.status + ST_BAD_FLAG, 1);
     __syncthreads();
+    // the block's count of each expert, and each warp's offset among the
+    // block's picks of it (16 counts loaded at a time before the running sum)
     for (int e = tid; e < E; e += THREADS) {
-        int t = 0;
-        for (int w = 0; w < NW; ++w) t += s.whist[w * E + e];
-        s.bcnt[e] = t;
-        p.hist[(long long)b * E + e] = t;
+        int run = 0;
+#pragma unroll
+        for (int w0 = 0; w0 < NW; w0 += 16) {
+            int v[16];
+#pragma unroll
+            for (int w = 0; w < 16; ++w) v[w] = s.whist[(w0 + w) * WS + e];
+#pragma unroll
+            for (int w = 0; w < 16; ++w) {
+                s.whist[(w0 + w) * WS + e] = run;
+                run += v[w];
+            }
+        }
+        s.bcnt[e] = run;
+        p.hist[(long long)b * E + e] = run;
+    }
+    __syncthreads();
+    unsigned* const barrier = reinterpret_cast<unsigned*>(p.status + ST_BARRIER1);
+    grid_arrive(barrier);
+
+    // expert-major slots of the block's picks; this needs only the block's
+    // own counts, so it runs while the other blocks finish their histograms
+    if (stash) {
+        int v1[1] = {tid < E ? s.bcnt[tid] : 0}, ex1[1], t1[1];
+        block_scan<1>(v1, ex1, t1, s.scratch);  // E <= THREADS
+        if (tid < E) {
+            // each warp's first slot of expert tid
+            s.bex[tid] = ex1[0];
+#pragma unroll
+            for (int w0 = 0; w0 < NW; w0 += 16) {
+                int v[16];
+#pragma unroll
+                for (int w = 0; w < 16; ++w) v[w] = s.whist[(w0 + w) * WS + tid];
+#pragma unroll
+                for (int w = 0; w < 16; ++w) s.whist[(w0 + w) * WS + tid] = v[w] + ex1[0];
+            }
+        }
+        __syncthreads();
+        for (unsigned base = wlo; base < whi; base += 32 * UNR) {
+            int v[UNR];
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                const unsigned q = base + u * 32 + lane;
+                v[u] = q < whi ? s.stash[q - clo] : -1;
+            }
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                if (v[u] >= 0) {
+                    const int e = v[u] & 1023;
+                    const int ql = (int)(base - clo) + u * 32 + lane;
+                    s.sorted[wh[e] + (v[u] >> 10)] = e | (ql << 10);
+                }
+            }
+        }
     }
 
-    if (!grid_wait(reinterpret_cast<unsigned*>(p.status + ST_BARRIER1),
-                   (unsigned)(G + p.barrier_extra), p.wait_ns, &wait_flag)) {
+    if (!grid_wait(barrier, (unsigned)(G + p.barrier_extra), p.wait_ns, &wait_flag)) {
         if (tid == 0) atomicMax(p.status + ST_STATUS, MOONEP_STATUS_TIMEOUT);
         return;
     }
@@ -561,75 +706,114 @@ __global__ void __launch_bounds__(THREADS, 1) plan_kernel(PlanParams p) {
             p.slot_expert[r * B + j] = j < nsl ? s.nzlist[nz0 + j] : -1;
     }
 
-    // per-warp running offsets: block offset + earlier warps' counts; and the
-    // per-expert placement tables
+    // the placement tables; on the expert-major path an entry is shifted by
+    // the offset sft from a slot of the block to the pick's position among
+    // all picks of its expert, so that the slot itself indexes the entry
     for (int e = tid; e < E; e += THREADS) {
-        int run = s.bpre[e];
-        for (int w = 0; w < NW; ++w) {
-            const int t = s.whist[w * E + e];
-            s.whist[w * E + e] = run;
-            run += t;
-        }
         const int first = (e / Er) * Er;
         const int k = s.kk[e];
-        s.tab[e] = make_int4(k, (e / Er) * p.C + (s.pk[e] - s.pk[first]), s.ose[e] - k, s.cnt[e]);
-        const int o = s.ov[e];
-        s.rng[e] = o > 0 ? upper_bound(s.sege_at, R, s.ose[e]) |
-                               (upper_bound(s.sege_at, R, s.ose[e] + o - 1) << 16)
-                         : 0;
+        const int sft = stash ? s.bpre[e] - s.bex[e] : 0;
+        s.tab[e] = make_int4(k - sft, (e / Er) * p.C + (s.pk[e] - s.pk[first]) + sft,
+                             s.ose[e] - k + sft, s.cnt[e] - sft);
+    }
+    if (!stash) {
+        // each warp's running offsets: the block's offset plus the warp's
+        // offset in the block
+        for (int i = tid; i < NW * E; i += THREADS) {
+            const int w = i / E, e = i - w * E;
+            s.whist[w * WS + e] += s.bpre[e];
+        }
     }
     for (int i = tid; i < R; i += THREADS) {
         const int rho = s.recv_at[i];
         s.rbase[i] = rho * p.C + s.kept[rho] - s.segs[rho];
     }
+    // the bucket width: the smallest power of two that covers the overflow
+    // stream (as long as the deficits' sum) in NBKT buckets; the last NBKT
+    // threads fill the buckets (the first E fill the tables above)
+    int sh = 0;
+    while (((long long)NBKT << sh) < (long long)s.osi[E]) ++sh;
+    if (tid >= THREADS - NBKT) {
+        const int i = tid - (THREADS - NBKT);
+        const int first = (int)((long long)i << sh);
+        const int last = (int)(((long long)(i + 1) << sh) - 1);
+        s.bkt[i] = upper_bound(s.sege_at, R, first) | (upper_bound(s.sege_at, R, last) << 16);
+    }
     __syncthreads();
 
     int internal = 0;
-    for (long long base = wlo; base < whi; base += 32 * UNR) {
-        const int nu = (int)min((long long)UNR, (whi - base + 31) / 32);  // warp-uniform
-        int ev[UNR], pos[UNR];
-        if (p.stash) {
-            // positions within the warp were found in phase A
+    if (stash) {
+        // the walk in expert-major order: consecutive threads place
+        // consecutive picks of one expert, whose rows are consecutive too
+        // (within a receiving segment), so the inverse map is written in runs;
+        // each pick's row goes to the stash, indexed by the pick
+        constexpr int WU = 4;  // slots per thread in flight
+        for (int i0 = tid; i0 < len; i0 += WU * THREADS) {
+            int v[WU];
 #pragma unroll
-            for (int u = 0; u < UNR; ++u) {
-                const long long q = base + u * 32 + lane;
-                const int v = q < whi ? s.stash[q - clo] : -1;
-                ev[u] = v >= 0 ? (v & 1023) : -1;
-                pos[u] = v >= 0 ? wh[v & 1023] + (v >> 10) : 0;
-            }
-        } else {
-            // picks not kept: read them again, match each row and advance the
-            // warp's running offsets row by row
-#pragma unroll
-            for (int u = 0; u < UNR; ++u) {
-                const long long q = base + u * 32 + lane;
-                ev[u] = q < whi ? __ldg(p.idx + q) : -1;
+            for (int u = 0; u < WU; ++u) {
+                const int i = i0 + u * THREADS;
+                v[u] = i < len ? s.sorted[i] : -1;
             }
 #pragma unroll
-            for (int u = 0; u < UNR; ++u) {
-                if (u < nu) {
-                    const int e = ev[u];
-                    const unsigned peers = __match_any_sync(0xffffffffu, e);
-                    const int run = e >= 0 ? wh[e] : 0;
-                    pos[u] = run + __popc(peers & lt_mask);
-                    __syncwarp();
-                    if (e >= 0 && lane == __ffs(peers) - 1) wh[e] = run + __popc(peers);
-                    __syncwarp();
+            for (int u = 0; u < WU; ++u) {
+                if (v[u] >= 0) {
+                    const int e = v[u] & 1023, ql = v[u] >> 10;
+                    const int pos = i0 + u * THREADS;  // the slot (entries are shifted)
+                    const int4 t = s.tab[e];
+                    const int dst = place(p, s, t, pos, sh);
+                    if (dst >= 0 && dst < p.P && pos < t.w) {
+                        p.src_of_row[dst] = (int)(clo + ql);
+                        s.stash[ql] = dst;
+                    } else {
+                        s.stash[ql] = -1;  // never expected: report, do not write
+                        internal = 1;
+                    }
                 }
             }
         }
+        __syncthreads();
+        for (int i0 = tid; i0 < len; i0 += WU * THREADS) {
+            int d[WU];
 #pragma unroll
-        for (int u = 0; u < UNR; ++u) {
-            const int e = ev[u];
-            if (u < nu && e >= 0) {
-                const long long q = base + u * 32 + lane;
-                const int4 t = s.tab[e];
-                const int dst = place(p, s, e, t, pos[u]);
-                if (dst >= 0 && dst < p.P && pos[u] < t.w) {
-                    p.dst_row[q] = dst;
-                    p.src_of_row[dst] = (int)q;
-                } else {
-                    internal = 1;  // never expected: report, do not write
+            for (int u = 0; u < WU; ++u) {
+                const int i = i0 + u * THREADS;
+                d[u] = i < len ? s.stash[i] : -1;
+            }
+#pragma unroll
+            for (int u = 0; u < WU; ++u)
+                if (d[u] >= 0) p.dst_row[clo + i0 + u * THREADS] = d[u];
+        }
+    } else {
+        // picks not kept: read them again and rank each row against the
+        // warp's running offsets.  Phase A checked every index; one that has
+        // changed since is reported, not placed.
+        for (unsigned base = wlo; base < whi; base += 32 * UNR) {
+            const int nu = (int)min((unsigned)UNR, (whi - base + 31) / 32);  // warp-uniform
+            int ev[UNR], pos[UNR];
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                const unsigned q = base + u * 32 + lane;
+                const int v = q < whi ? __ldg(p.idx + q) : -1;
+                ev[u] = v < E ? v : -1;
+                if (q < whi && (v < 0 || v >= E)) internal = 1;
+            }
+#pragma unroll
+            for (int u = 0; u < UNR; ++u)
+                if (u < nu) pos[u] = rank_row<MASK>(wh, wm, ev[u], lane, lt_mask, cand);
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                const int e = ev[u];
+                if (u < nu && e >= 0) {
+                    const unsigned q = base + u * 32 + lane;
+                    const int4 t = s.tab[e];
+                    const int dst = place(p, s, t, pos[u], sh);
+                    if (dst >= 0 && dst < p.P && pos[u] < t.w) {
+                        p.dst_row[q] = dst;
+                        p.src_of_row[dst] = (int)q;
+                    } else {
+                        internal = 1;  // never expected: report, do not write
+                    }
                 }
             }
         }
@@ -640,7 +824,7 @@ __global__ void __launch_bounds__(THREADS, 1) plan_kernel(PlanParams p) {
 struct DevInfo {
     int sms = 0;
     int max_smem_optin = 0;
-    size_t smem_set = 0;  // largest dynamic smem the kernel has been configured for
+    size_t smem_set[2] = {0, 0};  // largest dynamic smem each form has been configured for
 };
 
 DevInfo& dev_info() {
@@ -687,38 +871,45 @@ cudaError_t launch_plan(const PlanLaunch& a, cudaStream_t stream, const char** w
     p.wait_ns = a.wait_ns;
     p.barrier_extra = a.barrier_extra;
 
-    // Shared memory: the fixed part, then the pick stash (saves re-reading
-    // the picks from L2 in the walk) if it fits.
-    const size_t base_bytes = smem_ints(a.E, a.R) * 4;
-    const long long chunk = ((long long)p.P + G - 1) / G;
+    // Shared memory, the first layout that fits: ranking by mask words (else
+    // by match.any) and keeping the block's picks (the stash and the
+    // expert-major order: no second read and ranking of the picks, and the
+    // walk writes its rows in runs), then either alone, then neither.
     const size_t limit = (size_t)info.max_smem_optin - 1024;
+    const long long chunk = ((long long)p.P + G - 1) / G;
+    bool mask = false, keep = false;
+    const bool forms[4][2] = {{true, true}, {false, true}, {true, false}, {false, false}};
+    for (int f = 0; f < 4; ++f) {
+        mask = forms[f][0];
+        keep = forms[f][1];
+        if (smem_ints(a.E, a.R, mask, keep, chunk) * 4 <= limit) break;
+    }
     p.chunk = (int)chunk;
-    p.stash = base_bytes + (size_t)chunk * 4 <= limit;
-    const size_t smem = base_bytes + (size_t)chunk * 4 * p.stash;
+    p.stash = keep;
+    const size_t smem = smem_ints(a.E, a.R, mask, keep, chunk) * 4;
     if (smem > (size_t)info.max_smem_optin) {
         *why = "planner shared memory exceeds the device limit (E or R too large)";
         return cudaErrorInvalidValue;
     }
+    const void* kern = mask ? (const void*)plan_kernel<true> : (const void*)plan_kernel<false>;
     cudaError_t err;
-    if (smem > info.smem_set) {
-        err = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)smem);
+    if (smem > info.smem_set[mask]) {
+        err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (err != cudaSuccess) return err;
         int per_sm = 0;
-        err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, plan_kernel, THREADS, smem);
+        err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, THREADS, smem);
         if (err != cudaSuccess) return err;
         if (per_sm < 1) {
             *why = "planner block does not fit on an SM";
             return cudaErrorInvalidConfiguration;
         }
-        info.smem_set = smem;
+        info.smem_set[mask] = smem;
     }
     // status block: status, fail info, the wait counter and the bad-index flag
     err = cudaMemsetAsync(a.plan.status, 0, MOONEP_STATUS_WORDS * sizeof(int32_t), stream);
     if (err != cudaSuccess) return err;
     void* args[] = {&p};
-    return cudaLaunchCooperativeKernel((const void*)plan_kernel, dim3(G), dim3(THREADS), args, smem,
-                                       stream);
+    return cudaLaunchCooperativeKernel(kern, dim3(G), dim3(THREADS), args, smem, stream);
 }
 
 }  // namespace moonep

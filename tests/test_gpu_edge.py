@@ -89,6 +89,21 @@ def test_largest_E_and_R():
         _full_check(cfgd, idx, w, rule=rule, expert="identity")
 
 
+@pytest.mark.parametrize("R,S,E,K", [
+    (8, 40000, 512, 8),  # 2.56 M picks: ranked by mask words; too many picks per
+                         # block to keep in shared memory, so the walk reads and
+                         # ranks them again in (t, k) order
+    (8, 8192, 1024, 8),  # E = 1024 and 524 K picks: no room for the mask words
+                         # (match.any) nor for the picks
+])
+def test_planner_picks_not_kept(R, S, E, K):
+    cfgd = _cfg(R, S, E, K, 16, 64, alpha=0.8)
+    idx, w = wl.routing(cfgd, seed=3)
+    for rule in (0, 1, 2):  # rule 0 runs out of slots here; 1 and 2 place
+        out, o = _full_check(cfgd, idx, w, rule=rule, expert="scale")
+        assert (o["status"] == 0) == (rule > 0)
+
+
 def test_duplicate_picks_and_all_to_one():
     cfgd = _cfg(4, 64, 8, 4, 8, 16)
     idx = np.full((256, 4), 5, np.int32)  # every pick on one expert
