@@ -441,9 +441,9 @@ __device__ __forceinline__ int pack_pick(int e, int off) { return e | (off << 10
 //   and after the warp's barrier one read gives the whole group, so the rank
 //   does not depend on the order the atomics were carried out in.  The
 //   candidate (warp-uniform) stays while it holds 4 or more lanes of a row,
-//   else it becomes the expert of the lowest lane outside it: under a heavy
-//   skew it settles on the hot expert, whose lanes would otherwise all set
-//   bits in one word, one after another.
+//   else it becomes lane 0's expert in this row: under a heavy skew it soon
+//   settles on the hot expert, whose lanes would otherwise all set bits in
+//   one word, one after another.
 //   The group's lowest lane advances the count and clears the word (every
 //   word is zero between rows).  Top-k routing keeps the lanes sharing a word
 //   few: a token's k experts are distinct, so at most ceil(31 / k) + 1 lanes
@@ -458,10 +458,7 @@ __device__ __forceinline__ int rank_row(int* wh, unsigned* wm, int e, int lane, 
         const unsigned mc = __ballot_sync(0xffffffffu, e >= 0 && e == cand);
         const bool inc = (mc >> lane) & 1u;
         if (e >= 0 && !inc) atomicOr(wm + e, 1u << lane);
-        if (__popc(mc) < 4) {
-            const unsigned rest = __ballot_sync(0xffffffffu, e >= 0) & ~mc;
-            if (rest) cand = __shfl_sync(0xffffffffu, e, __ffs(rest) - 1);
-        }
+        if (__popc(mc) < 4) cand = __shfl_sync(0xffffffffu, e, 0);
         __syncwarp();
         m = inc ? mc : (e >= 0 ? wm[e] : 0u);
     } else {
@@ -514,7 +511,24 @@ __global__ void __launch_bounds__(THREADS, 1) plan_kernel(PlanParams p) {
     __syncthreads();
     int bad = 0;
     int cand = -1;  // the warp's candidate expert (ranking by masks)
-    for (unsigned base = wlo; base < whi; base += 32 * UNR) {
+    unsigned base = wlo;
+    // whole batches of UNR rows: every lane has a pick, no bounds checks
+    for (; base + 32 * UNR <= whi; base += 32 * UNR) {
+        int ev[UNR];
+#pragma unroll
+        for (int u = 0; u < UNR; ++u) ev[u] = __ldg(p.idx + base + u * 32 + lane);
+        const int qo = (int)(base - clo) + lane;
+#pragma unroll
+        for (int u = 0; u < UNR; ++u) {
+            const int e = ev[u];
+            const bool ok = (unsigned)e < (unsigned)E;
+            bad |= !ok;
+            const int off = rank_row<MASK>(wh, wm, ok ? e : -1, lane, lt_mask, cand);
+            if (stash) s.stash[qo + u * 32] = ok ? pack_pick(e, off) : -1;
+        }
+    }
+    // the last, partial batch
+    for (; base < whi; base += 32 * UNR) {
         int ev[UNR];
 #pragma unroll
         for (int u = 0; u < UNR; ++u) {
