@@ -145,6 +145,31 @@ def test_bad_index_reported_and_no_data_moved():
     assert me().plan_status(out["bufs"])[0] == me().STATUS_BAD_INDEX
 
 
+@pytest.fixture(scope="module")
+def many_picks():
+    cfgd = _cfg(8, 32768, 64, 8, 8, 16)  # 2.1 M picks: about 440 per warp
+    idx, _ = wl.routing(cfgd, seed=1)
+    return cfgd, idx
+
+
+@pytest.mark.parametrize("q,bad", [(0, 64), (1000, -1), (777_777, 1 << 20), (2_097_151, -64)])
+def test_bad_index_among_many_picks(many_picks, q, bad):
+    """At this size every warp ranks whole batches of 8 rows (no per-row
+    bounds checks) before its last, partial batch; an index outside [0, E) in
+    either is still reported."""
+    cfgd, idx = many_picks
+    m = me()
+    cfg = m.config_from(cfgd, 0)
+    bufs = m.PlanBuffers(cfg)
+    bad_idx = idx.copy()
+    bad_idx.reshape(-1)[q] = bad
+    m.plan(cfg, torch.from_numpy(bad_idx).cuda(), bufs)
+    assert m.plan_status(bufs)[0] == m.STATUS_BAD_INDEX
+    m.plan(cfg, torch.from_numpy(idx).cuda(), bufs)  # the same buffers, valid picks
+    o = oracle.plan(cfgd["R"], cfgd["S"], cfgd["E"], cfgd["K"], cfgd["B"], idx)
+    compare_plans(bufs.host(), o)
+
+
 def test_wait_that_runs_out_reports_timeout():
     """The planner's first grid-wide wait is told to expect one block more
     than exists; it gives up after the (short) wait limit, the plan reports
