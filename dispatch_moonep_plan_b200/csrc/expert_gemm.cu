@@ -29,10 +29,15 @@
 //    (32 columns each) fit the 512 columns; the last n-tile may be partial;
 //  - the fp32 accumulator lives in tensor memory; with 128-row tiles there
 //    are two buffers, so the epilogue of one tile overlaps the main loop of
-//    the next (the 256 x 256 and the fp8 tiles fill the 512 columns with one
-//    buffer, and their epilogue does not);
+//    the next.  The 256 x 256 tile fills the 512 columns with one buffer of
+//    two 128-row halves, which the epilogue frees one at a time: the next
+//    tile's first-half MMAs start once the first half is drained, while its
+//    second-half MMAs wait (holding their stages, at most all of them) for
+//    the second.  The fp8 tile's one buffer is not overlapped;
 //  - the epilogue reads 32 lanes x 32 columns per tcgen05.ld, rounds once to
-//    bf16 (round-to-nearest-even) and stores only the rows of the group.
+//    bf16 (round-to-nearest-even) and stores only the rows of the group; for
+//    bf16 rows each warp passes its 32 rows x 64 B through shared memory, so
+//    that one store covers 64 contiguous bytes of 8 rows.
 //
 // The tile list is built in each CTA from the plan: only the groups a plan
 // can fill are visited (rank r's E/R home experts and its B slots; every
@@ -89,6 +94,18 @@ __device__ __forceinline__ bool mbar_test(uint64_t* b, uint32_t parity) {
     uint32_t done;
     asm volatile(
         "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; "
+        "selp.u32 %0, 1, 0, p; }"
+        : "=r"(done)
+        : "r"(smem_u32(b)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Whether the phase of `parity` has completed, without suspending the thread.
+__device__ __forceinline__ bool mbar_peek(uint64_t* b, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2; "
         "selp.u32 %0, 1, 0, p; }"
         : "=r"(done)
         : "r"(smem_u32(b)), "r"(parity)
@@ -268,6 +285,9 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
     constexpr int NACC = (FP8A ? 2 * TN + 32 * STAGES : 2 * MT * TN) <= 512 ? 2 : 1;
     constexpr int ACOL = NACC * TN;
     constexpr int ACC_COLS = MT * TN;  // one accumulator: the MT halves side by side
+    // one accumulator of two halves: the epilogue frees each half on its own
+    // (tempty[h]), so the next tile's first half starts while the second drains
+    constexpr bool SPLIT = !FP8A && MT == 2 && NACC == 1;
     constexpr int TMEM_COLS = FP8A ? 512 : NACC * ACC_COLS;
     static_assert(NACC * ACC_COLS + (FP8A ? 32 * STAGES : 0) <= 512 && ACC_COLS <= 512,
                   "accumulators (and fp8 A stages) in the 512 tensor-memory columns");
@@ -303,6 +323,8 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
     const int G = p.E + p.B;      // groups per rank
     const int per = p.Er + p.B;   // groups a plan can fill per rank
     const int npairs = p.R * per;
+    // bf16 payload: the epilogue's row staging, [4 warps][32 rows][80 B]
+    uint8_t* estage = (uint8_t*)(((uintptr_t)(pre + npairs + 1) + 15) & ~(uintptr_t)15);
     const int ntn = (p.Hp + TN - 1) / TN;  // the last n-tile may be partial
     const int kblocks = p.H / BK;
 
@@ -452,8 +474,38 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
             int acc = 0;
             uint32_t acc_ph = 0;
             bool any = false;
+            // the MMAs of stage st (k-block kb) into the halves [h0, h1)
+            auto issue = [&](int st, int kb, int h0, int h1, int nsub, uint32_t d) {
+                const uint32_t a = smem_u32(smem + st * STAGE_BYTES);
+                const uint32_t b = a + STAGE_A;
+#pragma unroll
+                for (int ks = 0; ks < BK / 16; ++ks) {
+#pragma unroll
+                    for (int h = 0; h < MT; ++h) {
+                        if (h < h0) continue;
+                        if (h >= h1) break;
+#pragma unroll
+                        for (int sub = 0; sub < NSUB; ++sub) {
+                            if (sub >= nsub) break;
+                            // half h, sub-tile sub: columns h*TN + sub*BN.. of the
+                            // accumulator, A rows of half h, B chunks sub*BN/64..
+                            const uint32_t bsub = b + sub * (BN / 64) * 8192;
+                            if constexpr (FP8A)
+                                mma_bf16_tmem_a(d + sub * BN, tmem + ACOL + st * 32 + ks * 8,
+                                                sdesc(bsub + ks * 2048, 8192, 1024), idesc,
+                                                (kb | ks) ? 1u : 0u);
+                            else
+                                mma_bf16(d + h * TN + sub * BN,
+                                         sdesc(a + h * A_BYTES + ks * 32, 16, 1024),
+                                         sdesc(bsub + ks * 2048, 8192, 1024), idesc,
+                                         (kb | ks) ? 1u : 0u);
+                        }
+                    }
+                }
+            };
             for (int tile = blockIdx.x; tile < total && !abort_flag; tile += gridDim.x) {
-                if (!mbar_wait(&tempty[acc], acc_ph ^ 1, p.wait_ns, &abort_flag)) break;
+                // SPLIT: only half 0 needs to be drained to start the tile
+                if (!mbar_wait(&tempty[SPLIT ? 0 : acc], acc_ph ^ 1, p.wait_ns, &abort_flag)) break;
                 asm volatile("tcgen05.fence::after_thread_sync;");
                 const uint32_t d = tmem + acc * ACC_COLS;
                 // sub-tiles wholly past H' (a partial last n-tile), and halves
@@ -465,6 +517,21 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
                 const int grows = __ldg(p.cu + r_ * G + g_) - (g_ ? __ldg(p.cu + r_ * G + g_ - 1) : 0);
                 const int nhalf = min(MT, (grows - mt_ * TM + BM - 1) / BM);
                 bool ok = true;
+                // SPLIT: while the epilogue still drains half 1 of the last
+                // tile, this tile's half-1 MMAs wait and their stages stay
+                // held (at most all STAGES of them); then they are issued in
+                // k order and each stage is released
+                bool h1_free = !SPLIT;
+                int npend = 0, pend_s = 0, pend_kb = 0;
+                auto flush = [&]() {
+                    int ss = pend_s;
+                    for (int j = 0; j < npend; ++j) {
+                        issue(ss, pend_kb + j, 1, 2, nsub, d);
+                        mma_commit(&empty[ss]);
+                        if (++ss == STAGES) ss = 0;
+                    }
+                    npend = 0;
+                };
                 for (int kb = 0; kb < kblocks; ++kb) {
                     // the TMA loads landed; fp8: and the converter warps have
                     // widened A into the stage
@@ -474,39 +541,42 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
                         break;
                     }
                     asm volatile("tcgen05.fence::after_thread_sync;");
-                    const uint32_t a = smem_u32(smem + s * STAGE_BYTES);
-                    const uint32_t b = a + STAGE_A;
-#pragma unroll
-                    for (int ks = 0; ks < BK / 16; ++ks) {
-#pragma unroll
-                        for (int h = 0; h < MT; ++h) {
-                            if (h >= nhalf) break;
-#pragma unroll
-                            for (int sub = 0; sub < NSUB; ++sub) {
-                                if (sub >= nsub) break;
-                                // half h, sub-tile sub: columns h*TN + sub*BN.. of the
-                                // accumulator, A rows of half h, B chunks sub*BN/64..
-                                const uint32_t bsub = b + sub * (BN / 64) * 8192;
-                                if constexpr (FP8A)
-                                    mma_bf16_tmem_a(d + sub * BN, tmem + ACOL + s * 32 + ks * 8,
-                                                    sdesc(bsub + ks * 2048, 8192, 1024), idesc,
-                                                    (kb | ks) ? 1u : 0u);
-                                else
-                                    mma_bf16(d + h * TN + sub * BN,
-                                             sdesc(a + h * A_BYTES + ks * 32, 16, 1024),
-                                             sdesc(bsub + ks * 2048, 8192, 1024), idesc,
-                                             (kb | ks) ? 1u : 0u);
-                            }
-                        }
-                    }
+                    const bool defer = SPLIT && !h1_free && nhalf > 1;
+                    issue(s, kb, 0, defer ? 1 : nhalf, nsub, d);
                     any = true;
-                    mma_commit(&empty[s]);
+                    if (defer) {
+                        if (npend == 0) {
+                            pend_s = s;
+                            pend_kb = kb;
+                        }
+                        ++npend;
+                        bool freed = mbar_peek(&tempty[1], acc_ph ^ 1);
+                        if (!freed && npend == STAGES) {  // out of stages: wait for the drain
+                            if (!mbar_wait(&tempty[1], acc_ph ^ 1, p.wait_ns, &abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            freed = true;
+                        }
+                        if (freed) {
+                            h1_free = true;
+                            asm volatile("tcgen05.fence::after_thread_sync;");
+                            flush();
+                        }
+                    } else {
+                        mma_commit(&empty[s]);
+                    }
                     if (++s == STAGES) {
                         s = 0;
                         ph ^= 1;
                     }
                 }
                 if (!ok) break;
+                if (!h1_free) {  // SPLIT: take the drain's phase; issue what still waits
+                    if (!mbar_wait(&tempty[1], acc_ph ^ 1, p.wait_ns, &abort_flag)) break;
+                    asm volatile("tcgen05.fence::after_thread_sync;");
+                    flush();
+                }
                 mma_commit(&tfull[acc]);
                 if (++acc == NACC) {
                     acc = 0;
@@ -533,7 +603,15 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
             asm volatile("tcgen05.fence::after_thread_sync;");
 #pragma unroll 1
             for (int h = 0; h < MT; ++h) {
-                if (mt * TM + h * BM >= ghi - glo) break;  // half past the group (warp-uniform)
+                if (mt * TM + h * BM >= ghi - glo) {  // half past the group (warp-uniform)
+                    if constexpr (SPLIT) {
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&tempty[h]);
+                        continue;
+                    } else {
+                        break;
+                    }
+                }
                 const int row_in = mt * TM + h * BM + q * 32 + lane;
                 const bool valid = glo + row_in < ghi;
                 uint16_t* yrow = p.y + (size_t)(r * p.C + glo + row_in) * p.Hp + nt * TN;
@@ -554,7 +632,33 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
                           "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
                         : "r"(tbase + c0));
                     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-                    if (valid) {
+                    if constexpr (!FP8A) {
+                        // the warp's 32 rows x 64 B go through shared memory
+                        // (80-byte row pitch: no bank conflicts either way), so
+                        // that each store writes 64 contiguous bytes of 8 rows
+                        // instead of 16 bytes of 32 rows
+                        uint8_t* wst = estage + q * (32 * 80);
+#pragma unroll
+                        for (int j = 0; j < 32; j += 8) {
+                            uint4 o;
+                            o.x = pack_bf16x2(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+                            o.y = pack_bf16x2(__uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+                            o.z = pack_bf16x2(__uint_as_float(v[j + 4]), __uint_as_float(v[j + 5]));
+                            o.w = pack_bf16x2(__uint_as_float(v[j + 6]), __uint_as_float(v[j + 7]));
+                            *reinterpret_cast<uint4*>(wst + lane * 80 + (j / 8) * 16) = o;
+                        }
+                        __syncwarp();
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int rr = 8 * i + (lane >> 2), k = lane & 3;  // row, 16-B piece
+                            const uint4 o = *reinterpret_cast<const uint4*>(wst + rr * 80 + k * 16);
+                            const int ri = mt * TM + h * BM + q * 32 + rr;
+                            if (glo + ri < ghi)
+                                *reinterpret_cast<uint4*>(p.y + (size_t)(r * p.C + glo + ri) * p.Hp +
+                                                          nt * TN + c0 + k * 8) = o;
+                        }
+                        __syncwarp();
+                    } else if (valid) {
 #pragma unroll
                         for (int j = 0; j < 32; j += 8) {
                             uint4 o;
@@ -566,10 +670,17 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
                         }
                     }
                 }
+                if constexpr (SPLIT) {  // this half is drained: the next tile may use it
+                    asm volatile("tcgen05.fence::before_thread_sync;");
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tempty[h]);
+                }
             }
-            asm volatile("tcgen05.fence::before_thread_sync;");
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[acc]);
+            if constexpr (!SPLIT) {
+                asm volatile("tcgen05.fence::before_thread_sync;");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[acc]);
+            }
             if (++acc == NACC) {
                 acc = 0;
                 acc_ph ^= 1;
@@ -725,11 +836,12 @@ bool encode_2d(CUtensorMap* m, const void* base, CUtensorMapDataType type, uint6
 
 // alignment slack + stages + e4m3 ring + barriers (3 per stage, 2 per e4m3
 // slot, 2 + 2 accumulator, drain, never) + TMEM address + per-warp sums +
-// the m-tile prefix
+// the m-tile prefix + (bf16 payload) the epilogue's row staging
 size_t smem_bytes(int bn, int stages, int npairs, bool fp8a, int a8_slots = 2, int mt = 1) {
     return 1024 + (size_t)stages * ((fp8a ? 0 : mt * A_BYTES) + BK * bn * 2) +
            (fp8a ? a8_slots * A8_BYTES : 0) +
-           (size_t)(3 * stages + 2 * a8_slots + 6) * 8 + 8 + 32 * 4 + (size_t)(npairs + 1) * 4;
+           (size_t)(3 * stages + 2 * a8_slots + 6) * 8 + 8 + 32 * 4 + (size_t)(npairs + 1) * 4 +
+           (fp8a ? 0 : 16 + 4 * 32 * 80);
 }
 
 template <int BN, int STAGES, bool FP8A, int CW = 8, int A8_SLOTS = 2, int NSUB = 1, int MT = 1>
