@@ -35,9 +35,9 @@
 //    second-half MMAs wait (holding their stages, at most all of them) for
 //    the second.  The fp8 tile's one buffer is not overlapped;
 //  - the epilogue reads 32 lanes x 32 columns per tcgen05.ld, rounds once to
-//    bf16 (round-to-nearest-even) and stores only the rows of the group; for
-//    bf16 rows each warp passes its 32 rows x 64 B through shared memory, so
-//    that one store covers 64 contiguous bytes of 8 rows.
+//    bf16 (round-to-nearest-even) and stores only the rows of the group;
+//    each warp passes its 32 rows x 64 B through shared memory, so that one
+//    store covers 64 contiguous bytes of 8 rows.
 //
 // The tile list is built in each CTA from the plan: only the groups a plan
 // can fill are visited (rank r's E/R home experts and its B slots; every
@@ -286,7 +286,10 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
     constexpr int ACOL = NACC * TN;
     constexpr int ACC_COLS = MT * TN;  // one accumulator: the MT halves side by side
     // one accumulator of two halves: the epilogue frees each half on its own
-    // (tempty[h]), so the next tile's first half starts while the second drains
+    // (tempty[h]), so the next tile's first half starts while the second
+    // drains.  (Splitting the fp8 tile's two column sub-tiles the same way was
+    // slower: the deferred MMAs hold the widened A stages, and the converter
+    // warps wait for them.)
     constexpr bool SPLIT = !FP8A && MT == 2 && NACC == 1;
     constexpr int TMEM_COLS = FP8A ? 512 : NACC * ACC_COLS;
     static_assert(NACC * ACC_COLS + (FP8A ? 32 * STAGES : 0) <= 512 && ACC_COLS <= 512,
@@ -323,7 +326,7 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
     const int G = p.E + p.B;      // groups per rank
     const int per = p.Er + p.B;   // groups a plan can fill per rank
     const int npairs = p.R * per;
-    // bf16 payload: the epilogue's row staging, [4 warps][32 rows][80 B]
+    // the epilogue's row staging, [4 warps][32 rows][80 B]
     uint8_t* estage = (uint8_t*)(((uintptr_t)(pre + npairs + 1) + 15) & ~(uintptr_t)15);
     const int ntn = (p.Hp + TN - 1) / TN;  // the last n-tile may be partial
     const int kblocks = p.H / BK;
@@ -612,9 +615,7 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
                         break;
                     }
                 }
-                const int row_in = mt * TM + h * BM + q * 32 + lane;
-                const bool valid = glo + row_in < ghi;
-                uint16_t* yrow = p.y + (size_t)(r * p.C + glo + row_in) * p.Hp + nt * TN;
+                uint8_t* wst = estage + q * (32 * 80);  // this warp's row staging
                 const uint32_t tbase = tmem + acc * ACC_COLS + h * TN + ((uint32_t)(q * 32) << 16);
 #pragma unroll 1
                 for (int c0 = 0; c0 < TN; c0 += 32) {
@@ -632,43 +633,30 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
                           "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
                         : "r"(tbase + c0));
                     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-                    if constexpr (!FP8A) {
-                        // the warp's 32 rows x 64 B go through shared memory
-                        // (80-byte row pitch: no bank conflicts either way), so
-                        // that each store writes 64 contiguous bytes of 8 rows
-                        // instead of 16 bytes of 32 rows
-                        uint8_t* wst = estage + q * (32 * 80);
+                    // the warp's 32 rows x 64 B go through shared memory (80-byte
+                    // row pitch: no bank conflicts either way), so that each
+                    // store writes 64 contiguous bytes of 8 rows instead of 16
+                    // bytes of 32 rows; only rows of the group are stored
 #pragma unroll
-                        for (int j = 0; j < 32; j += 8) {
-                            uint4 o;
-                            o.x = pack_bf16x2(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
-                            o.y = pack_bf16x2(__uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
-                            o.z = pack_bf16x2(__uint_as_float(v[j + 4]), __uint_as_float(v[j + 5]));
-                            o.w = pack_bf16x2(__uint_as_float(v[j + 6]), __uint_as_float(v[j + 7]));
-                            *reinterpret_cast<uint4*>(wst + lane * 80 + (j / 8) * 16) = o;
-                        }
-                        __syncwarp();
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int rr = 8 * i + (lane >> 2), k = lane & 3;  // row, 16-B piece
-                            const uint4 o = *reinterpret_cast<const uint4*>(wst + rr * 80 + k * 16);
-                            const int ri = mt * TM + h * BM + q * 32 + rr;
-                            if (glo + ri < ghi)
-                                *reinterpret_cast<uint4*>(p.y + (size_t)(r * p.C + glo + ri) * p.Hp +
-                                                          nt * TN + c0 + k * 8) = o;
-                        }
-                        __syncwarp();
-                    } else if (valid) {
-#pragma unroll
-                        for (int j = 0; j < 32; j += 8) {
-                            uint4 o;
-                            o.x = pack_bf16x2(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
-                            o.y = pack_bf16x2(__uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
-                            o.z = pack_bf16x2(__uint_as_float(v[j + 4]), __uint_as_float(v[j + 5]));
-                            o.w = pack_bf16x2(__uint_as_float(v[j + 6]), __uint_as_float(v[j + 7]));
-                            *reinterpret_cast<uint4*>(yrow + c0 + j) = o;
-                        }
+                    for (int j = 0; j < 32; j += 8) {
+                        uint4 o;
+                        o.x = pack_bf16x2(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+                        o.y = pack_bf16x2(__uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+                        o.z = pack_bf16x2(__uint_as_float(v[j + 4]), __uint_as_float(v[j + 5]));
+                        o.w = pack_bf16x2(__uint_as_float(v[j + 6]), __uint_as_float(v[j + 7]));
+                        *reinterpret_cast<uint4*>(wst + lane * 80 + (j / 8) * 16) = o;
                     }
+                    __syncwarp();
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int rr = 8 * i + (lane >> 2), k = lane & 3;  // row, 16-B piece
+                        const uint4 o = *reinterpret_cast<const uint4*>(wst + rr * 80 + k * 16);
+                        const int ri = mt * TM + h * BM + q * 32 + rr;
+                        if (glo + ri < ghi)
+                            *reinterpret_cast<uint4*>(p.y + (size_t)(r * p.C + glo + ri) * p.Hp +
+                                                      nt * TN + c0 + k * 8) = o;
+                    }
+                    __syncwarp();
                 }
                 if constexpr (SPLIT) {  // this half is drained: the next tile may use it
                     asm volatile("tcgen05.fence::before_thread_sync;");
@@ -836,12 +824,12 @@ bool encode_2d(CUtensorMap* m, const void* base, CUtensorMapDataType type, uint6
 
 // alignment slack + stages + e4m3 ring + barriers (3 per stage, 2 per e4m3
 // slot, 2 + 2 accumulator, drain, never) + TMEM address + per-warp sums +
-// the m-tile prefix + (bf16 payload) the epilogue's row staging
+// the m-tile prefix + the epilogue's row staging
 size_t smem_bytes(int bn, int stages, int npairs, bool fp8a, int a8_slots = 2, int mt = 1) {
     return 1024 + (size_t)stages * ((fp8a ? 0 : mt * A_BYTES) + BK * bn * 2) +
            (fp8a ? a8_slots * A8_BYTES : 0) +
            (size_t)(3 * stages + 2 * a8_slots + 6) * 8 + 8 + 32 * 4 + (size_t)(npairs + 1) * 4 +
-           (fp8a ? 0 : 16 + 4 * 32 * 80);
+           16 + 4 * 32 * 80;
 }
 
 template <int BN, int STAGES, bool FP8A, int CW = 8, int A8_SLOTS = 2, int NSUB = 1, int MT = 1>
