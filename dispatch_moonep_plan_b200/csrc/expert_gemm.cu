@@ -11,8 +11,9 @@
 // for sm_100a:
 //
 //  - one persistent CTA per SM: warp 0 issues TMA loads, one thread of warp 1
-//    issues tcgen05.mma, warps 2-9 drain the accumulator (two per TMEM lane
-//    quarter, each taking half of the columns: 320 threads);
+//    issues tcgen05.mma, 8 warps drain the accumulator (two per TMEM lane
+//    quarter, each taking half of the columns): warps 2-9 for bf16 rows (320
+//    threads), warps 2-5 and 15-18 for fp8 rows (608 threads);
 //  - bf16 payload: tile 256 rows x 256 columns when H' % 256 == 0 (else 128
 //    x BN, BN = 256 or 128), k-block 64: A = two 128 x 64 bf16 blocks of the
 //    dispatched rows (K-major), B = 64 x 256 of the weight row (H'
@@ -67,11 +68,12 @@ constexpr int BK = 64;
 constexpr int A_BYTES = BM * BK * 2;   // 16 KiB of bf16 A per stage
 constexpr int A8_BYTES = BM * BK;      // 8 KiB of e4m3 A per k-block (fp8 payload)
 // fp8 payload: one more warp loads the e4m3 tiles and CW warps widen them
-// epilogue warps of the bf16 payload: two per TMEM lane quarter, each taking
-// half of a tile's columns (the fp8 payload keeps one per quarter)
-constexpr int EWB = 8;
+// 8 epilogue warps: two per TMEM lane quarter, each taking half of a tile's
+// columns.  bf16 payload: warps 2-9; fp8 payload: warps 2-5 and, after the
+// e4m3 producer (warp 6) and the CW converter warps, the last 4
+constexpr int EPI_WARPS = 8;
 template <bool FP8A, int CW>
-__host__ __device__ constexpr int threads_for() { return FP8A ? (7 + CW) * 32 : (2 + EWB) * 32; }
+__host__ __device__ constexpr int threads_for() { return FP8A ? (7 + CW + 4) * 32 : (2 + EPI_WARPS) * 32; }
 // dynamic shared memory a CTA may ask for: the 227 KiB opt-in limit less
 // room for the kernel's static shared variables
 constexpr int SMEM_LIMIT = 227 * 1024 - 256;
@@ -348,7 +350,7 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
-            mbar_init(&tempty[a], FP8A ? 4 : EWB);
+            mbar_init(&tempty[a], EPI_WARPS);
         }
         mbar_init(drain, 1);
         mbar_init(never, 1);
@@ -595,11 +597,13 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
                 mbar_drain(drain, 0, p.wait_ns);
             }
         }
-    } else if (warp < 2 + (FP8A ? 4 : EWB)) {  // epilogue: warp w reads TMEM lanes 32*(w % 4) .. +31
+    } else if ((warp >= 2 && warp < (FP8A ? 6 : 2 + EPI_WARPS)) || (FP8A && warp >= 7 + CW)) {
+        // epilogue: warp w reads TMEM lanes 32*(w % 4) .. +31, and half of the
+        // tile's columns
         const int q = warp & 3;
-        constexpr int CP = FP8A ? 1 : EWB / 4;  // warps per lane quarter
-        const int cpart = (warp - 2) >> 2;      // which part of the tile's columns
-        const int c_lo = cpart * (TN / CP), c_hi = c_lo + TN / CP;
+        const int eord = (FP8A && warp >= 7 + CW) ? 4 + (warp - 7 - CW) : warp - 2;  // 0..7
+        const int cpart = eord >> 2;
+        const int c_lo = cpart * (TN / 2), c_hi = c_lo + TN / 2;
         int acc = 0;
         uint32_t acc_ph = 0;
         for (int tile = blockIdx.x; tile < total && !abort_flag; tile += gridDim.x) {
@@ -622,7 +626,7 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
                         break;
                     }
                 }
-                uint8_t* wst = estage + (warp - 2) * (32 * 80);  // this warp's row staging
+                uint8_t* wst = estage + eord * (32 * 80);  // this warp's row staging
                 const uint32_t tbase = tmem + acc * ACC_COLS + h * TN + ((uint32_t)(q * 32) << 16);
 #pragma unroll 1
                 for (int c0 = c_lo; c0 < c_hi; c0 += 32) {
@@ -836,7 +840,7 @@ size_t smem_bytes(int bn, int stages, int npairs, bool fp8a, int a8_slots = 2, i
     return 1024 + (size_t)stages * ((fp8a ? 0 : mt * A_BYTES) + BK * bn * 2) +
            (fp8a ? a8_slots * A8_BYTES : 0) +
            (size_t)(3 * stages + 2 * a8_slots + 6) * 8 + 8 + 32 * 4 + (size_t)(npairs + 1) * 4 +
-           16 + (fp8a ? 4 : EWB) * 32 * 80;
+           16 + EPI_WARPS * 32 * 80;
 }
 
 template <int BN, int STAGES, bool FP8A, int CW = 8, int A8_SLOTS = 2, int NSUB = 1, int MT = 1>
