@@ -13,14 +13,14 @@
 // that every block is resident and the grid-wide wait cannot deadlock):
 //   A. each block owns a contiguous run of picks, each warp a contiguous part
 //      of it; every warp ranks its picks 32 at a time in (t, k) order: the
-//      lanes holding the same expert are found (one ballot for lane 0's
-//      expert, lane-mask words in shared memory for the rest, or match.any
-//      when the words do not fit), and the group's lowest lane advances the
-//      warp's count of that expert; count before the row plus the lane's rank
-//      in its group is the pick's position among the warp's picks of the
-//      expert, kept beside the pick in shared memory.  One warp per expert
-//      then scans the 32 warps' counts: the block's row hist[block][e] and
-//      each warp's offset within the block.
+//      lanes holding the same expert are found (one ballot for the warp's
+//      candidate expert, lane-mask words in shared memory for the rest, or
+//      match.any when the words do not fit), and the group's lowest lane
+//      advances the warp's count of that expert; count before the row plus
+//      the lane's rank in its group is the pick's position among the warp's
+//      picks of the expert, kept beside the pick in shared memory.  One
+//      thread per expert then runs over the 32 warps' counts: the block's row
+//      hist[block][e] and each warp's offset within the block.
 //   -- one grid-wide wait; while it lasts, each block sorts its own picks
 //      into expert-major order in shared memory (slot = the block's prefix
 //      over experts + the warp's offset + the position in the warp) --
@@ -117,8 +117,8 @@ struct Smem {
                   //         in the warp << 10; later each pick's destination row
 };
 
-// Row stride of the per-warp arrays: odd, so that the 32 warps' entries of
-// one expert lie in 32 different banks.
+// Row stride of the per-warp arrays: E rounded up to an odd count of words
+// (rows of neighbouring warps start in different banks).
 __host__ __device__ inline int warp_stride(int E) { return E | 1; }
 
 __host__ __device__ inline size_t smem_ints(int E, int R, bool mask, bool stash, long long chunk) {
