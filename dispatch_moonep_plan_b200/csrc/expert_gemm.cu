@@ -265,7 +265,7 @@ struct GemmArgs {
     int debug_stall;  // epilogue waits on a barrier nothing completes
 };
 
-template <int BN, int STAGES, bool FP8A, int CW, int A8_SLOTS, int NSUB, int MT>
+template <int BN, int STAGES, bool FP8A, int CW, int A8_SLOTS, int NSUB, int MT, bool STG>
 __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
     expert_gemm_kernel(const __grid_constant__ CUtensorMap tmX,
                        const __grid_constant__ CUtensorMap tmW, GemmArgs p) {
@@ -626,7 +626,8 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
                         break;
                     }
                 }
-                uint8_t* wst = estage + eord * (32 * 80);  // this warp's row staging
+                uint8_t* wst = estage + eord * (32 * 80);  // this warp's row staging (STG)
+                const int row_in = mt * TM + h * BM + q * 32 + lane;  // this lane's row (!STG)
                 const uint32_t tbase = tmem + acc * ACC_COLS + h * TN + ((uint32_t)(q * 32) << 16);
 #pragma unroll 1
                 for (int c0 = c_lo; c0 < c_hi; c0 += 32) {
@@ -644,30 +645,46 @@ __global__ void __launch_bounds__(threads_for<FP8A, CW>(), 1)
                           "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
                         : "r"(tbase + c0));
                     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-                    // the warp's 32 rows x 64 B go through shared memory (80-byte
-                    // row pitch: no bank conflicts either way), so that each
-                    // store writes 64 contiguous bytes of 8 rows instead of 16
-                    // bytes of 32 rows; only rows of the group are stored
+                    if constexpr (!STG) {  // each lane stores its own row's 64 B
+                        if (glo + row_in < ghi) {
+                            uint16_t* yrow =
+                                p.y + (size_t)(r * p.C + glo + row_in) * p.Hp + nt * TN + c0;
 #pragma unroll
-                    for (int j = 0; j < 32; j += 8) {
-                        uint4 o;
-                        o.x = pack_bf16x2(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
-                        o.y = pack_bf16x2(__uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
-                        o.z = pack_bf16x2(__uint_as_float(v[j + 4]), __uint_as_float(v[j + 5]));
-                        o.w = pack_bf16x2(__uint_as_float(v[j + 6]), __uint_as_float(v[j + 7]));
-                        *reinterpret_cast<uint4*>(wst + lane * 80 + (j / 8) * 16) = o;
-                    }
-                    __syncwarp();
+                            for (int j = 0; j < 32; j += 8) {
+                                uint4 o;
+                                o.x = pack_bf16x2(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+                                o.y = pack_bf16x2(__uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+                                o.z = pack_bf16x2(__uint_as_float(v[j + 4]), __uint_as_float(v[j + 5]));
+                                o.w = pack_bf16x2(__uint_as_float(v[j + 6]), __uint_as_float(v[j + 7]));
+                                *reinterpret_cast<uint4*>(yrow + j) = o;
+                            }
+                        }
+                    } else {
+                        // the warp's 32 rows x 64 B go through shared memory (80-byte
+                        // row pitch: no bank conflicts either way), so that each
+                        // store writes 64 contiguous bytes of 8 rows instead of 16
+                        // bytes of 32 rows; only rows of the group are stored
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int rr = 8 * i + (lane >> 2), k = lane & 3;  // row, 16-B piece
-                        const uint4 o = *reinterpret_cast<const uint4*>(wst + rr * 80 + k * 16);
-                        const int ri = mt * TM + h * BM + q * 32 + rr;
-                        if (glo + ri < ghi)
-                            *reinterpret_cast<uint4*>(p.y + (size_t)(r * p.C + glo + ri) * p.Hp +
-                                                      nt * TN + c0 + k * 8) = o;
+                        for (int j = 0; j < 32; j += 8) {
+                            uint4 o;
+                            o.x = pack_bf16x2(__uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+                            o.y = pack_bf16x2(__uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+                            o.z = pack_bf16x2(__uint_as_float(v[j + 4]), __uint_as_float(v[j + 5]));
+                            o.w = pack_bf16x2(__uint_as_float(v[j + 6]), __uint_as_float(v[j + 7]));
+                            *reinterpret_cast<uint4*>(wst + lane * 80 + (j / 8) * 16) = o;
+                        }
+                        __syncwarp();
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int rr = 8 * i + (lane >> 2), k = lane & 3;  // row, 16-B piece
+                            const uint4 o = *reinterpret_cast<const uint4*>(wst + rr * 80 + k * 16);
+                            const int ri = mt * TM + h * BM + q * 32 + rr;
+                            if (glo + ri < ghi)
+                                *reinterpret_cast<uint4*>(p.y + (size_t)(r * p.C + glo + ri) * p.Hp +
+                                                          nt * TN + c0 + k * 8) = o;
+                        }
+                        __syncwarp();
                     }
-                    __syncwarp();
                 }
                 if constexpr (SPLIT) {  // this half is drained: the next tile may use it
                     asm volatile("tcgen05.fence::before_thread_sync;");
@@ -836,14 +853,16 @@ bool encode_2d(CUtensorMap* m, const void* base, CUtensorMapDataType type, uint6
 // alignment slack + stages + e4m3 ring + barriers (3 per stage, 2 per e4m3
 // slot, 2 + 2 accumulator, drain, never) + TMEM address + per-warp sums +
 // the m-tile prefix + the epilogue's row staging
-size_t smem_bytes(int bn, int stages, int npairs, bool fp8a, int a8_slots = 2, int mt = 1) {
+size_t smem_bytes(int bn, int stages, int npairs, bool fp8a, int a8_slots = 2, int mt = 1,
+                  bool stg = true) {
     return 1024 + (size_t)stages * ((fp8a ? 0 : mt * A_BYTES) + BK * bn * 2) +
            (fp8a ? a8_slots * A8_BYTES : 0) +
            (size_t)(3 * stages + 2 * a8_slots + 6) * 8 + 8 + 32 * 4 + (size_t)(npairs + 1) * 4 +
-           16 + EPI_WARPS * 32 * 80;
+           (stg ? 16 + EPI_WARPS * 32 * 80 : 0);
 }
 
-template <int BN, int STAGES, bool FP8A, int CW = 8, int A8_SLOTS = 2, int NSUB = 1, int MT = 1>
+template <int BN, int STAGES, bool FP8A, int CW = 8, int A8_SLOTS = 2, int NSUB = 1, int MT = 1,
+          bool STG = true>
 cudaError_t launch_variant(const CUtensorMap& x, const CUtensorMap& w, const GemmArgs& a,
                            size_t smem, int grid, cudaStream_t s) {
     static std::mutex mu;
@@ -854,13 +873,13 @@ cudaError_t launch_variant(const CUtensorMap& x, const CUtensorMap& w, const Gem
     {
         std::lock_guard<std::mutex> lock(mu);
         if (dev < 0 || dev >= 64 || set[dev] < smem) {
-            e = cudaFuncSetAttribute(expert_gemm_kernel<BN, STAGES, FP8A, CW, A8_SLOTS, NSUB, MT>,
+            e = cudaFuncSetAttribute(expert_gemm_kernel<BN, STAGES, FP8A, CW, A8_SLOTS, NSUB, MT, STG>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return e;
             if (dev >= 0 && dev < 64) set[dev] = smem;
         }
     }
-    expert_gemm_kernel<BN, STAGES, FP8A, CW, A8_SLOTS, NSUB, MT>
+    expert_gemm_kernel<BN, STAGES, FP8A, CW, A8_SLOTS, NSUB, MT, STG>
         <<<grid, threads_for<FP8A, CW>(), smem, s>>>(x, w, a);
     return cudaGetLastError();
 }
@@ -877,8 +896,11 @@ constexpr int FP8_A8 = 4;
 // the fp8 kernel's configuration, or the smallest bf16 one
 bool expert_gemm_fits(const moonep_config& c) {
     const int np = expert_gemm_npairs(c);
-    return (c.payload == MOONEP_PAYLOAD_FP8 ? smem_bytes(FP8_TN, FP8_STAGES, np, true, FP8_A8)
-                                            : smem_bytes(128, 3, np, false)) <= (size_t)SMEM_LIMIT;
+    // the smallest layout of each payload: fp8 without the epilogue's row
+    // staging (E + R*B up to 9216 pairs fits either way)
+    return (c.payload == MOONEP_PAYLOAD_FP8
+                ? smem_bytes(FP8_TN, FP8_STAGES, np, true, FP8_A8, 1, false)
+                : smem_bytes(128, 3, np, false)) <= (size_t)SMEM_LIMIT;
 }
 
 cudaError_t launch_expert_gemm(const moonep_config& c, const moonep_plan_t& p, const void* x,
@@ -912,10 +934,16 @@ cudaError_t launch_expert_gemm(const moonep_config& c, const moonep_plan_t& p, c
     a.wait_ns = current_wait_limit_ns();
     a.debug_stall = current_barrier_extra() != 0;
     const int grid = device_sm_count();
-    if (fp8)  // 128 x 384 tiles (two MMAs of N = 192 per widened A block): one
-              // accumulator and 3 A stages in the 512 TMEM columns
-        return launch_variant<192, FP8_STAGES, true, 8, FP8_A8, FP8_TN / 192>(
-            tx, tw, a, smem_bytes(FP8_TN, FP8_STAGES, np, true, FP8_A8), grid, s);
+    if (fp8) {  // 128 x 384 tiles (two MMAs of N = 192 per widened A block): one
+                // accumulator and 3 A stages in the 512 TMEM columns; the
+                // epilogue's row staging when it fits beside the m-tile prefix
+        const size_t s1 = smem_bytes(FP8_TN, FP8_STAGES, np, true, FP8_A8, 1, true);
+        if (s1 <= (size_t)SMEM_LIMIT)
+            return launch_variant<192, FP8_STAGES, true, 8, FP8_A8, FP8_TN / 192, 1, true>(
+                tx, tw, a, s1, grid, s);
+        return launch_variant<192, FP8_STAGES, true, 8, FP8_A8, FP8_TN / 192, 1, false>(
+            tx, tw, a, smem_bytes(FP8_TN, FP8_STAGES, np, true, FP8_A8, 1, false), grid, s);
+    }
     if (c.Hp % 256 == 0) {
 #ifndef GEMM_MT1
         // 256 x 256 tiles (two m-tiles per B block), one accumulator

@@ -299,7 +299,9 @@ int moonep_expert_standin(const moonep_config* cfg, const moonep_plan_t* plan, c
  * not exist (every rank holds exactly C rows); only the groups a plan can
  * fill are read: rank r's E/R home experts and its B slots.
  * Requires H % 64 == 0, Hp % 128 == 0, R*(E+B)*H < 2^31, recv_scale for
- * the fp8 payload and 16-byte aligned pointers (else INVALID_ARG).  Does
+ * the fp8 payload and 16-byte aligned pointers (else INVALID_ARG).  The
+ * kernel keeps one entry per (rank, group) pair, E + R*B of them, in shared
+ * memory; every configuration within the MOONEP_MAX_* bounds fits.  Does
  * nothing when the plan's status is not OK; a device wait that runs out sets
  * MOONEP_STATUS_TIMEOUT (out is then partly written). */
 int moonep_expert_gemm(const moonep_config* cfg, const moonep_plan_t* plan, const void* recv,

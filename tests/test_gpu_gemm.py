@@ -396,6 +396,18 @@ def test_fp8_random_shapes_and_ragged():
     assert done >= 5
 
 
+def test_fp8_many_pairs_without_epilogue_staging():
+    """E + R*B = 128 + 128*64 = 8320 (rank, group) pairs: the m-tile prefix
+    leaves no room for the epilogue's row staging next to the fp8 stages, so
+    the kernel stores each lane's row directly; same results."""
+    done = 0
+    for rule in (1, 2):
+        if _run_fp8(_small(128, 8, 128, 2, 64, 128, 128, alpha=1.2), rule=rule, seed=0,
+                    integer=True) is not None:
+            done += 1
+    assert done >= 1
+
+
 def test_fp8_wait_that_runs_out_reports_timeout():
     """The same stalled epilogue with the converter warps running: every role,
     converters included, stops at the wait limit and the status is TIMEOUT;
