@@ -104,6 +104,23 @@ def test_planner_picks_not_kept(R, S, E, K):
         assert (o["status"] == 0) == (rule > 0)
 
 
+@pytest.mark.parametrize("alpha", [0.0, 3.0])
+def test_planner_one_pick_per_token_few_experts(alpha):
+    """K = 1 and E = 8 over 2.1 M picks: a row of 32 picks spans 32 tokens, so
+    up to 32 lanes hold one expert (the mask words' worst case) in whole
+    batches of rows, and the candidate expert keeps changing (alpha 0) or
+    stays on the hot one (alpha 3)."""
+    cfgd = _cfg(8, 262144, 8, 1, 8, 16, alpha=alpha)
+    idx, _ = wl.routing(cfgd, seed=5)
+    m = me()
+    for rule in (1, 2):
+        cfg = m.config_from(cfgd, rule)
+        bufs = m.PlanBuffers(cfg)
+        m.plan(cfg, torch.from_numpy(idx).cuda(), bufs)
+        o = oracle.plan(cfgd["R"], cfgd["S"], cfgd["E"], cfgd["K"], cfgd["B"], idx, rule=rule)
+        compare_plans(bufs.host(), o)
+
+
 def test_duplicate_picks_and_all_to_one():
     cfgd = _cfg(4, 64, 8, 4, 8, 16)
     idx = np.full((256, 4), 5, np.int32)  # every pick on one expert
